@@ -1,0 +1,12 @@
+"""Plain float64 CPU oracle for exact long-context attention.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The product path (the
+C-ABI library and its Python binding) never imports, links or runs anything
+here, and this package imports nothing from the product path.
+
+Modules:
+  attention  exact attention rows, single-token decode, log-sum-exp merge
+  fp8        E4M3 code table from the format definition
+  stream     exact-cover check of a (query block, key chunk) task list
+"""
