@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+Headline: causal GQA prefill, batch 2, 32 query / 8 KV heads, head dim 128, 8192 tokens,
+bf16 in / fp32 accumulate, in TFLOP/s (algorithmic FLOPs: the causal half only).  The same
+JSON line carries the split-KV decode workloads (ragged bf16 64K-128K cache; FP8 E4M3 cache,
+32768 tokens) in KV GB/s, each against the measured roofline, the oracle timed on the host
+cores, and an end-to-end number through host buffers.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--stream]
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU (independent
+replicas: weak scaling, no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from exact_long_context_tmem_b200 import inputs as I  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s & decode KV GB/s at 1 B200, as fraction of roofline"
+HEADLINE = "prefill_b2_h32g8_d128_s8192"
+DECODE_WORKLOADS = ("decode_b4_h32g8_d128_ragged64k_128k", "decode_fp8_b16_h32g8_d128_t32768")
+STREAM = "stream_b1_h32g8_d128_s1m_chunk64k"
+L2_BYTES = 126 * 10**6
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        self.dev = device_index
+
+    def start(self):
+        try:
+            ident = None
+            try:
+                ident = str(torch.cuda.get_device_properties(self.dev).uuid)
+                if not ident.startswith("GPU-"):
+                    ident = "GPU-" + ident
+            except Exception:  # noqa: BLE001
+                ident = str(self.dev)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", ident], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:  # noqa: BLE001
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:  # noqa: BLE001
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workloads
+
+def prefill_flops(w):
+    # causal: row i sees i+1 keys; QK^T and PV are 2*D FLOPs per (row, key) each
+    pairs = w.S * (w.S + 1) // 2 if w.causal else w.S * w.T
+    return 4.0 * w.D * w.B * w.Hq * pairs
+
+
+def decode_bytes(w, lens):
+    tok = int(lens.sum())
+    per_tok = w.Hkv * w.D * (1 if w.kv_fp8 else 2) * 2
+    if w.kv_fp8:
+        per_tok += w.Hkv * 4 * 2  # k and v scales
+    qo = w.B * w.Hq * w.D * 2 * 2 + w.B * w.Hq * 4
+    return tok * per_tok + qo
+
+
+def bench_prefill(w, steps, warmup, world, dev, pk):
+    from exact_long_context_tmem_b200 import attn as A
+
+    q, k, v = I.prefill_inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty((w.B, w.S, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        A.attn_prefill(qd, kd, vd, causal=True, o=o, lse=lse)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index or 0)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t0.record()
+    for i in range(steps):
+        ev[i][0].record()
+        A.attn_prefill(qd, kd, vd, causal=True, o=o, lse=lse)
+        ev[i][1].record()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = prefill_flops(w)
+
+    # end to end: pinned host Q/K/V in, O and LSE back, every step
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        A.attn_prefill(qd, kd, vd, causal=True, o=o, lse=lse)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    for _ in range(max(1, warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, steps // 2)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = (q.numel() + k.numel() + v.numel()) * 2
+    d2h = o.numel() * 2 + lse.numel() * 4
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    return {
+        "total_ms": total_ms, "ms_per_step": total_ms / steps, "launch_ms": launch_ms, "flops": flops,
+        "tflops": flops * world / (total_ms / steps * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": None,
+                     "peak_kind": f"bf16 dense, burst, {pk['source']}",
+                     "frac_of_sustained": (round(achieved / pk["bf16_tflops_sustained"], 4)
+                                           if pk.get("bf16_tflops_sustained") else None)},
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks, "launches": steps,
+    }
+
+
+def bench_decode(name, steps, warmup, world, dev, pk):
+    from exact_long_context_tmem_b200 import attn as A
+
+    w = I.WORKLOADS[name]
+    d = I.decode_inputs(w)
+    lens = d["kv_lens"]
+    qd, ld = d["q"].to(dev), lens.to(dev)
+    if w.kv_fp8:
+        kd, vd = d["k_codes"].to(dev), d["v_codes"].to(dev)
+        ks, vs = d["k_scale"].to(dev), d["v_scale"].to(dev)
+    else:
+        kd, vd = d["k"].to(dev), d["v"].to(dev)
+        ks = vs = None
+    Tmax = d["Tmax"]
+    o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    nbytes = A.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, Tmax)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    splits = A.attn_decode_num_splits(w.B, w.Hq, w.Hkv, w.D, Tmax)
+
+    def step():
+        A.attn_decode_splitkv(qd, kd, vd, ld, k_scale=ks, v_scale=vs, o=o, lse=lse, ws=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    call_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    nb = decode_bytes(w, lens)
+    gbs = nb / (call_ms * 1e-3) / 1e9
+    return {"workload": name, "value": round(gbs * world, 1), "unit": "GB/s", "ms_per_step": round(call_ms, 4),
+            "splits": splits, "kv_tokens": int(lens.sum()), "bytes_per_step": nb,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": None,
+                         "timed": "split kernel + merge kernel (one API call)"},
+            "launches": steps * (2 if splits > 1 else 1)}
+
+
+def bench_stream(dev, pk):
+    from exact_long_context_tmem_b200 import attn as A
+
+    w = I.WORKLOADS[STREAM]
+    g = I.generator(w.seed)
+    shape_q = (w.B, w.S, w.Hq, w.D)
+    shape_kv = (w.B, w.S, w.Hkv, w.D)
+    q = I.randn_bf16(shape_q, g, out=torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True))
+    k = I.randn_bf16(shape_kv, g, out=torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True))
+    v = I.randn_bf16(shape_kv, g, out=torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True))
+    o = torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)
+    lse = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, pin_memory=True)
+    _, _, st = A.attn_chunked_stream(q, k, v, causal=True, chunk_tokens=w.chunk_tokens, budget_bytes=w.budget_bytes,
+                                     o_h=o, lse_h=lse)
+    flops = prefill_flops(w)
+    return {"workload": STREAM, "value": round(flops / (st.ms_total * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "ms_total": round(st.ms_total, 1), "q_block": st.plan.q_block, "kv_chunk": st.plan.kv_chunk,
+            "tasks": st.plan.n_tasks, "device_bytes": st.plan.device_bytes,
+            "h2d_GBps": round(st.h2d_bytes / (st.ms_total * 1e-3) / 1e9, 2),
+            "d2h_GBps": round(st.d2h_bytes / (st.ms_total * 1e-3) / 1e9, 2),
+            "h2d_bytes": st.h2d_bytes, "d2h_bytes": st.d2h_bytes}
+
+
+# ------------------------------------------------------------------ oracle (CPU baseline)
+
+def host_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:  # noqa: BLE001
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(w, n_rows, seed=4242):
+    """Time the float64 oracle on n_rows sampled query rows (all batches and heads) of the
+    prefill workload; returns (TFLOP/s of the sample, seconds, rows)."""
+    from oracle import attention as O
+
+    q, k, v = I.prefill_inputs(w)
+    rows = I.sample_rows(w.S, n_rows, seed=seed)
+    t = time.perf_counter()
+    O.attention(q, k, v, scale=w.scale, causal=True, rows=rows)
+    dt = time.perf_counter() - t
+    flops = sum(4.0 * w.D * (r + 1) for r in rows) * w.B * w.Hq
+    return flops / dt / 1e12, dt, rows
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--stream", action="store_true", help="also run the 1M-token streamed prefill")
+    ap.add_argument("--cpu-rows", type=int, default=128)
+    args = ap.parse_args()
+    w = I.WORKLOADS[HEADLINE]
+    config = {"workload": HEADLINE, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
+              "seq_len": w.S, "causal": True, "io": "bf16 Q/K/V/O, fp32 LSE",
+              "l2": "per step 192 MiB of inputs + 130 MiB of outputs > 126 MB L2; no flush",
+              "parallelism": f"replicas x{args.gpus}"}
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cores = host_threads()
+        vals = []
+        n_rows = max(4, args.cpu_rows // 8)
+        for i in range(args.warmup + args.steps):
+            tf, dt, rows = oracle_sample(w, n_rows, seed=9000 + i)
+            if i >= args.warmup:
+                vals.append((tf, dt))
+        value = statistics.mean(v for v, _ in vals)
+        line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 * statistics.mean(d for _, d in vals), 1),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic N(0,1), seeded", "config": config, "impl": "reference",
+                "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                 "sample": f"{n_rows} sampled query rows x {w.B} batch x {w.Hq} heads per step"},
+                "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    world, rank, local = dist_init(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from exact_long_context_tmem_b200 import attn as A
+    A.lib()
+    pk = peaks()
+    pre = bench_prefill(w, args.steps, args.warmup, world, dev, pk)
+    dec = []
+    if not args.no_decode:
+        for name in DECODE_WORKLOADS:
+            dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk))
+    st, site = A.attn_device_status(reset=True)
+    if st != 0:
+        raise SystemExit(f"device status {st} at wait site {site}")
+    stream = bench_stream(dev, pk) if args.stream and rank == 0 else None
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, dt, rows = oracle_sample(w, args.cpu_rows)
+        cpu = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
+               "sample": f"{len(rows)} sampled query rows x {w.B} batch x {w.Hq} heads ({dt:.1f} s)"}
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(pre["tflops"], 2), "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["ms_per_step"], 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic N(0,1), seeded", "config": config, "roofline": pre["roofline"],
+                "cpu_baseline": cpu, "e2e": pre["e2e"], "clocks": pre["clocks"], "gpu_launches": pre["launches"],
+                "decode": dec, "stream": stream}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,251 @@
+"""Thin ctypes binding of libattn.so (include/attn.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module only
+allocates output tensors with PyTorch, passes raw pointers, sizes and the current CUDA
+stream, and turns status codes into exceptions.  There is no fallback: if the library or
+a GPU is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn.so")
+
+ATTN_OK = 0
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "budget", 5: "timeout",
+          6: "injected"}
+ATTN_BF16, ATTN_FP8_E4M3, ATTN_F32 = 0, 1, 2
+
+EXPORTS = [
+    "attn_prefill", "attn_decode_workspace_bytes", "attn_decode_num_splits", "attn_decode_splitkv",
+    "attn_merge_lse", "attn_stream_plan", "attn_stream_task", "attn_chunked_stream", "attn_status_string",
+    "attn_last_cuda_error", "attn_device_status", "attn_set_wait_limit_ns", "attn_debug_wait_probe",
+    "attn_debug_inject",
+]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} (status {status})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int),
+                ("scale", ctypes.c_float)]
+
+
+class StreamPlan(ctypes.Structure):
+    _fields_ = [("q_block", ctypes.c_longlong), ("kv_chunk", ctypes.c_longlong), ("n_tasks", ctypes.c_longlong),
+                ("device_bytes", ctypes.c_longlong)]
+
+
+class StreamStats(ctypes.Structure):
+    _fields_ = [("plan", StreamPlan), ("h2d_bytes", ctypes.c_longlong), ("d2h_bytes", ctypes.c_longlong),
+                ("ms_total", ctypes.c_double), ("ms_compute", ctypes.c_double)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn.so (built in-tree by exact_long_context_tmem_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_long_context_tmem_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, ll, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t, ctypes.c_float
+    L.attn_prefill.argtypes = [vp, vp, vp, vp, i, vp, Dims, i, i, i, ll, ll, vp]
+    L.attn_prefill.restype = i
+    L.attn_decode_workspace_bytes.argtypes = [Dims, i, i]
+    L.attn_decode_workspace_bytes.restype = sz
+    L.attn_decode_num_splits.argtypes = [Dims, i, i]
+    L.attn_decode_num_splits.restype = i
+    L.attn_decode_splitkv.argtypes = [vp, vp, vp, i, vp, vp, vp, i, Dims, i, vp, vp, vp, sz, vp]
+    L.attn_decode_splitkv.restype = i
+    L.attn_merge_lse.argtypes = [vp, vp, i, ll, i, vp, i, vp, i, vp]
+    L.attn_merge_lse.restype = i
+    L.attn_stream_plan.argtypes = [Dims, ll, i, ll, sz, ctypes.POINTER(StreamPlan)]
+    L.attn_stream_plan.restype = i
+    L.attn_stream_task.argtypes = [ctypes.POINTER(StreamPlan), ll, i, ll, ctypes.POINTER(ll), ctypes.POINTER(ll)]
+    L.attn_stream_task.restype = i
+    L.attn_chunked_stream.argtypes = [vp, vp, vp, vp, vp, Dims, ll, i, ll, sz, vp, vp, ctypes.POINTER(StreamStats)]
+    L.attn_chunked_stream.restype = i
+    L.attn_status_string.argtypes = [i]
+    L.attn_status_string.restype = ctypes.c_char_p
+    L.attn_last_cuda_error.argtypes = []
+    L.attn_last_cuda_error.restype = i
+    L.attn_device_status.argtypes = [i, ctypes.POINTER(i)]
+    L.attn_device_status.restype = i
+    L.attn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    L.attn_set_wait_limit_ns.restype = i
+    L.attn_debug_wait_probe.argtypes = [ctypes.c_ulonglong]
+    L.attn_debug_wait_probe.restype = i
+    L.attn_debug_inject.argtypes = [i, ll]
+    L.attn_debug_inject.restype = i
+    _ = f
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str):
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dims(B, Hq, Hkv, D, scale):
+    return Dims(int(B), int(Hq), int(Hkv), int(D), float(scale))
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("device tensors expected (the library runs on the GPU only)")
+
+
+def attn_prefill(q, k, v, *, causal: bool = True, scale: float | None = None, q_pos0: int = 0, kv_pos0: int = 0,
+                 o=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True, stream=None):
+    """q [B,S,Hq,D], k/v [B,T,Hkv,D] bf16 CUDA tensors -> (o [B,S,Hq,D], lse [B,S,Hq] float32)."""
+    _need_cuda(q, k, v)
+    B, S, Hq, D = q.shape
+    T, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if o is None:
+        o = torch.empty((B, S, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
+    od = ATTN_F32 if o.dtype == torch.float32 else ATTN_BF16
+    st = lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), od, _ptr(lse), _dims(B, Hq, Hkv, D, scale), S, T,
+                            int(bool(causal)), int(q_pos0), int(kv_pos0), _stream(stream))
+    _check(st, "attn_prefill")
+    return o, lse
+
+
+def attn_decode_workspace_bytes(B, Hq, Hkv, D, Tmax, num_splits=0, scale=1.0) -> int:
+    return int(lib().attn_decode_workspace_bytes(_dims(B, Hq, Hkv, D, scale), int(Tmax), int(num_splits)))
+
+
+def attn_decode_num_splits(B, Hq, Hkv, D, Tmax, num_splits=0, scale=1.0) -> int:
+    return int(lib().attn_decode_num_splits(_dims(B, Hq, Hkv, D, scale), int(Tmax), int(num_splits)))
+
+
+def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: float | None = None,
+                        num_splits: int = 0, o=None, lse=None, ws=None, want_lse: bool = True, stream=None):
+    """q [B,Hq,D] bf16; k/v [B,Tmax,Hkv,D] bf16 or uint8 E4M3 codes (+ float32 scales [B,Tmax,Hkv]);
+    kv_lens int32 [B] on the device -> (o [B,Hq,D] bf16, lse [B,Hq] float32)."""
+    _need_cuda(q, k, v, kv_lens, k_scale, v_scale)
+    B, Hq, D = q.shape
+    Tmax, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    fp8 = k.dtype in (torch.uint8, torch.float8_e4m3fn)
+    dims = _dims(B, Hq, Hkv, D, scale)
+    if o is None:
+        o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = int(lib().attn_decode_workspace_bytes(dims, int(Tmax), int(num_splits)))
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().attn_decode_splitkv(_ptr(q), _ptr(k), _ptr(v), ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(k_scale),
+                                   _ptr(v_scale), _ptr(kv_lens), int(Tmax), dims, int(num_splits), _ptr(o),
+                                   _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
+    _check(st, "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_merge_lse(o_parts, lse_parts, *, o_out=None, lse_out=None, accumulate: bool = False,
+                   out_dtype=torch.float32, stream=None):
+    """o_parts float32 [P,R,D], lse_parts float32 [P,R] -> (o_out [R,D], lse_out [R])."""
+    _need_cuda(o_parts, lse_parts, o_out, lse_out)
+    P, R, D = o_parts.shape
+    if o_out is None:
+        o_out = torch.empty((R, D), dtype=out_dtype, device=o_parts.device)
+    if lse_out is None:
+        lse_out = torch.empty((R,), dtype=torch.float32, device=o_parts.device)
+    od = ATTN_F32 if o_out.dtype == torch.float32 else ATTN_BF16
+    st = lib().attn_merge_lse(_ptr(o_parts), _ptr(lse_parts), int(P), int(R), int(D), _ptr(o_out), od,
+                              _ptr(lse_out), int(bool(accumulate)), _stream(stream))
+    _check(st, "attn_merge_lse")
+    return o_out, lse_out
+
+
+def attn_stream_plan(B, Hq, Hkv, D, S, *, causal=True, chunk_tokens=0, budget_bytes=16 * 10**9, scale=None):
+    plan = StreamPlan()
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    st = lib().attn_stream_plan(_dims(B, Hq, Hkv, D, scale), int(S), int(bool(causal)), int(chunk_tokens),
+                                int(budget_bytes), ctypes.byref(plan))
+    _check(st, "attn_stream_plan")
+    return plan
+
+
+def attn_stream_task(plan: StreamPlan, S: int, causal: bool, idx: int):
+    q0, k0 = ctypes.c_longlong(), ctypes.c_longlong()
+    st = lib().attn_stream_task(ctypes.byref(plan), int(S), int(bool(causal)), int(idx), ctypes.byref(q0),
+                                ctypes.byref(k0))
+    _check(st, "attn_stream_task")
+    return q0.value, k0.value
+
+
+def attn_chunked_stream(q_h, k_h, v_h, *, causal=True, chunk_tokens=0, budget_bytes=16 * 10**9, scale=None,
+                        o_h=None, lse_h=None, want_lse=True, compute_stream=None, copy_stream=None):
+    """Host (ideally pinned) bf16 q_h [B,S,Hq,D], k_h/v_h [B,S,Hkv,D] -> host (o_h, lse_h, stats)."""
+    for t in (q_h, k_h, v_h):
+        if t.is_cuda:
+            raise ValueError("attn_chunked_stream takes host tensors")
+    B, S, Hq, D = q_h.shape
+    Hkv = k_h.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if o_h is None:
+        o_h = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, pin_memory=True)
+    if lse_h is None and want_lse:
+        lse_h = torch.empty((B, S, Hq), dtype=torch.float32, pin_memory=True)
+    stats = StreamStats()
+    cs = None if compute_stream is None else _stream(compute_stream)
+    xs = None if copy_stream is None else _stream(copy_stream)
+    st = lib().attn_chunked_stream(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(o_h), _ptr(lse_h),
+                                   _dims(B, Hq, Hkv, D, scale), int(S), int(bool(causal)), int(chunk_tokens),
+                                   int(budget_bytes), cs, xs, ctypes.byref(stats))
+    _check(st, "attn_chunked_stream")
+    return o_h, lse_h, stats
+
+
+def attn_device_status(reset: bool = False):
+    site = ctypes.c_int(0)
+    st = lib().attn_device_status(int(bool(reset)), ctypes.byref(site))
+    return st, site.value
+
+
+def attn_set_wait_limit_ns(ns: int):
+    _check(lib().attn_set_wait_limit_ns(int(ns)), "attn_set_wait_limit_ns")
+
+
+def attn_debug_wait_probe(limit_ns: int) -> int:
+    return int(lib().attn_debug_wait_probe(int(limit_ns)))
+
+
+def attn_debug_inject(what: int, nth: int):
+    _check(lib().attn_debug_inject(int(what), int(nth)), "attn_debug_inject")
+
+
+def attn_status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()

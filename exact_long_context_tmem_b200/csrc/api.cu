@@ -1,0 +1,396 @@
+// Host side of libattn.so: argument validation, TMA tensor maps, launch configuration and
+// the status/diagnostic entry points.  Every device kernel of the library is compiled in
+// this one translation unit, so the device status word exists once per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "decode.cuh"
+#include "merge.cuh"
+#include "prefill.cuh"
+
+namespace attn {
+
+static thread_local int t_last_cuda_error = 0;
+
+static attn_status_t cuda_fail(cudaError_t e) {
+  t_last_cuda_error = (int)e;
+  return ATTN_ERR_CUDA;
+}
+
+#define ATTN_CUDA(call)                          \
+  do {                                           \
+    cudaError_t e_ = (call);                     \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// ---------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D tiled map over a row-major [d3][d2][d1][d0] tensor, 128-byte swizzle, zero fill out of bounds.
+static attn_status_t make_map_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                                 const uint64_t dims[4], const uint32_t box[4]) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t gdim[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gstride[3] = {dims[0] * elem_bytes, dims[0] * dims[1] * elem_bytes,
+                           dims[0] * dims[1] * dims[2] * elem_bytes};
+  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = (int)r;
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename K>
+static attn_status_t ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  ATTN_CUDA(cudaGetDevice(&dev));
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done_mask.load(std::memory_order_acquire) & bit) return ATTN_OK;
+  ATTN_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return ATTN_OK;
+}
+
+static bool dims_ok(const attn_dims_t& d) {
+  return d.B >= 0 && d.Hq > 0 && d.Hkv > 0 && d.Hq % d.Hkv == 0 && d.D > 0 && std::isfinite(d.scale) &&
+         d.scale > 0.f;
+}
+
+static constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- prefill
+
+template <int D>
+static attn_status_t launch_prefill(const void* q, const void* k, const void* v, void* o, int o_f32, float* lse,
+                                    const attn_dims_t& d, int S, int T, int causal, long long q_pos0,
+                                    long long kv_pos0, cudaStream_t stream) {
+  using C = PrefillCfg<D>;
+  static std::atomic<uint64_t> smem_done{0};
+  attn_status_t st = ensure_smem(prefill_fwd_sm100<D>, C::SMEM_BYTES, smem_done);
+  if (st != ATTN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  const uint64_t dq[4] = {(uint64_t)D, (uint64_t)d.Hq, (uint64_t)S, (uint64_t)d.B};
+  const uint64_t dk[4] = {(uint64_t)D, (uint64_t)d.Hkv, (uint64_t)T, (uint64_t)d.B};
+  const uint32_t box[4] = {64, 1, 128, 1};
+  if ((st = make_map_4d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dq, box)) != ATTN_OK) return st;
+  if ((st = make_map_4d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box)) != ATTN_OK) return st;
+  if ((st = make_map_4d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box)) != ATTN_OK) return st;
+  PrefillParams p{};
+  p.B = d.B;
+  p.Hq = d.Hq;
+  p.Hkv = d.Hkv;
+  p.D = D;
+  p.S = S;
+  p.T = T;
+  p.G = d.Hq / d.Hkv;
+  p.causal = causal ? 1 : 0;
+  p.q_pos0 = q_pos0;
+  p.kv_pos0 = kv_pos0;
+  p.scale_log2 = d.scale * kLog2e;
+  p.n_qtiles = (S + 127) / 128;
+  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+  p.n_head_units = p.pair_heads ? d.Hq / 2 : d.Hq;
+  p.n_q_units = p.pair_heads ? p.n_qtiles : (p.n_qtiles + 1) / 2;
+  const long long items = (long long)d.B * p.n_head_units * p.n_q_units;
+  if (items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  p.n_items = (int)items;
+  p.o = o;
+  p.o_f32 = o_f32;
+  p.lse = lse;
+  prefill_fwd_sm100<D><<<p.n_items, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  ATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+// ---------------------------------------------------------------- decode planning
+
+static int decode_splits(const attn_dims_t& d, int Tmax, int requested) {
+  if (Tmax <= 0) return 1;
+  const int max_splits = (Tmax + 127) / 128;
+  int P = requested;
+  if (P <= 0) {
+    // One CTA per SM at a time (shared memory); aim for about four waves of CTAs, with every
+    // split at least 2048 tokens so the per-CTA set-up stays small next to its stream.
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long units = (long long)std::max(d.B, 1) * d.Hkv;
+    P = (int)std::max(1LL, (4LL * sms + units - 1) / units);
+    P = std::min(P, std::max(1, Tmax / 2048));
+  }
+  P = std::min(P, max_splits);
+  // Round the split length up to whole tiles, then recompute how many splits cover Tmax.
+  const int per = ((Tmax + P - 1) / P + 127) / 128 * 128;
+  return (Tmax + per - 1) / per;
+}
+
+static int decode_split_tokens(int Tmax, int P) {
+  if (Tmax <= 0) return 128;
+  return ((Tmax + P - 1) / P + 127) / 128 * 128;
+}
+
+static size_t decode_ws_bytes(const attn_dims_t& d, int P) {
+  if (P <= 1) return 0;
+  const size_t rows = (size_t)P * d.B * d.Hq;
+  return rows * d.D * sizeof(float) + rows * sizeof(float) + 256;
+}
+
+template <bool FP8>
+static attn_status_t launch_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
+                                   const int* kv_lens, int Tmax, const attn_dims_t& d, int P, int split_tokens,
+                                   void* o, float* lse, void* ws, cudaStream_t stream) {
+  using C = DecodeCfg<FP8>;
+  static std::atomic<uint64_t> smem_done{0};
+  attn_status_t st = ensure_smem(decode_split_sm100<FP8>, C::SMEM_BYTES, smem_done);
+  if (st != ATTN_OK) return st;
+  CUtensorMap mk, mv;
+  // With Tmax == 0 every split is empty and no map is read; it still needs a valid base and extent.
+  const uint64_t dk[4] = {128, (uint64_t)d.Hkv, (uint64_t)std::max(Tmax, 1), (uint64_t)d.B};
+  const void* kb = Tmax > 0 ? k : q;
+  const void* vb = Tmax > 0 ? v : q;
+  if (FP8) {
+    const uint32_t box[4] = {128, 1, 128, 1};
+    if ((st = make_map_4d(&mk, kb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dk, box)) != ATTN_OK) return st;
+    if ((st = make_map_4d(&mv, vb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dk, box)) != ATTN_OK) return st;
+  } else {
+    const uint32_t box[4] = {64, 1, 128, 1};
+    if ((st = make_map_4d(&mk, kb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box)) != ATTN_OK) return st;
+    if ((st = make_map_4d(&mv, vb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box)) != ATTN_OK) return st;
+  }
+  DecodeParams p{};
+  p.B = d.B;
+  p.Hq = d.Hq;
+  p.Hkv = d.Hkv;
+  p.G = d.Hq / d.Hkv;
+  p.Tmax = Tmax;
+  p.split_tokens = split_tokens;
+  p.n_splits = P;
+  p.scale_log2 = d.scale * kLog2e;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.k_scale = ks;
+  p.v_scale = vs;
+  p.kv_lens = kv_lens;
+  float* ws_f = reinterpret_cast<float*>(ws);
+  const size_t rows = (size_t)P * d.B * d.Hq;
+  p.o_part = P > 1 ? ws_f : nullptr;
+  p.lse_part = P > 1 ? ws_f + rows * 128 : nullptr;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  dim3 grid(P, d.Hkv, d.B);
+  decode_split_sm100<FP8><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, p);
+  ATTN_CUDA(cudaGetLastError());
+  if (P > 1) {
+    MergeParams mp{};
+    mp.o_parts = p.o_part;
+    mp.lse_parts = p.lse_part;
+    mp.P = P;
+    mp.R = (long long)d.B * d.Hq;
+    mp.o_out = o;
+    mp.o_f32 = 0;
+    mp.lse_out = lse;
+    mp.accumulate = 0;
+    const long long blocks = (mp.R + 7) / 8;
+    merge_lse_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(mp);
+    ATTN_CUDA(cudaGetLastError());
+  }
+  return ATTN_OK;
+}
+
+// ---------------------------------------------------------------- diagnostics
+
+__global__ void wait_probe_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, SITE_PROBE);  // nothing arrives: runs out and records
+  __syncthreads();
+}
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_BUDGET: return "device budget too small for the smallest plan";
+    case ATTN_ERR_TIMEOUT: return "a kernel wait ran out of time";
+    case ATTN_ERR_INJECTED: return "injected failure";
+  }
+  return "unknown status";
+}
+
+int attn_last_cuda_error(void) { return t_last_cuda_error; }
+
+attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o, attn_dtype_t o_dtype, float* lse,
+                           attn_dims_t dims, int S, int T, int causal, long long q_pos0, long long kv_pos0,
+                           void* stream) {
+  if (!dims_ok(dims) || S < 0 || T < 0 || q_pos0 < 0 || kv_pos0 < 0) return ATTN_ERR_INVALID_ARG;
+  if (o_dtype != ATTN_BF16 && o_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  if (dims.B == 0 || S == 0) return ATTN_OK;
+  if (!q || !o || (T > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || (T > 0 && (!aligned16(k) || !aligned16(v))) || (lse && !aligned4(lse)))
+    return ATTN_ERR_INVALID_ARG;
+  if (dims.D != 64 && dims.D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (T == 0) {
+    // No keys: every row is empty.  O = 0, LSE = -inf, written by the merge kernel with no parts.
+    MergeParams mp{};
+    mp.P = 0;
+    mp.R = (long long)dims.B * S * dims.Hq;
+    mp.o_out = o;
+    mp.o_f32 = o_dtype == ATTN_F32;
+    mp.lse_out = lse;
+    mp.accumulate = 0;
+    const long long blocks = (mp.R + 7) / 8;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dims.D == 128) merge_lse_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(mp);
+    else merge_lse_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(mp);
+    ATTN_CUDA(cudaGetLastError());
+    return ATTN_OK;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int f32 = o_dtype == ATTN_F32;
+  if (dims.D == 128) return launch_prefill<128>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st);
+  return launch_prefill<64>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st);
+}
+
+int attn_decode_num_splits(attn_dims_t dims, int Tmax, int num_splits) {
+  if (!dims_ok(dims) || Tmax < 0) return 0;
+  return decode_splits(dims, Tmax, num_splits);
+}
+
+size_t attn_decode_workspace_bytes(attn_dims_t dims, int Tmax, int num_splits) {
+  if (!dims_ok(dims) || Tmax < 0) return 0;
+  return decode_ws_bytes(dims, decode_splits(dims, Tmax, num_splits));
+}
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                  const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax,
+                                  attn_dims_t dims, int num_splits, void* o, float* lse, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  if (!dims_ok(dims) || Tmax < 0 || num_splits < 0 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
+  if (kv_dtype != ATTN_BF16 && kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (dims.B == 0) return ATTN_OK;
+  if (!q || !o || !kv_lens || (Tmax > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  const bool fp8 = kv_dtype == ATTN_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr) || fp8 != (v_scale != nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned4(kv_lens) || (lse && !aligned4(lse))) return ATTN_ERR_INVALID_ARG;
+  if (Tmax > 0 && (!aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
+  if (fp8 && (!aligned4(k_scale) || !aligned4(v_scale))) return ATTN_ERR_INVALID_ARG;
+  if (dims.D != 128 || dims.Hq / dims.Hkv > 16) return ATTN_ERR_UNSUPPORTED;
+  if (dims.B > 65535 || dims.Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  const int P = decode_splits(dims, Tmax, num_splits);
+  const size_t need = decode_ws_bytes(dims, P);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int per = decode_split_tokens(Tmax, P);
+  if (fp8) return launch_decode<true>(q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st);
+  return launch_decode<false>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st);
+}
+
+attn_status_t attn_merge_lse(const float* o_parts, const float* lse_parts, int P, long long R, int D, void* o_out,
+                             attn_dtype_t o_dtype, float* lse_out, int accumulate, void* stream) {
+  if (P < 0 || R < 0 || (P == 0 && !accumulate)) return ATTN_ERR_INVALID_ARG;
+  if (o_dtype != ATTN_BF16 && o_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  if (accumulate && (o_dtype != ATTN_F32 || !lse_out)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (R == 0) return ATTN_OK;
+  if (!o_out || (P > 0 && (!o_parts || !lse_parts))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_out) || (P > 0 && (!aligned16(o_parts) || !aligned4(lse_parts))) || (lse_out && !aligned4(lse_out)))
+    return ATTN_ERR_INVALID_ARG;
+  const long long blocks = (R + 7) / 8;
+  if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  MergeParams mp{};
+  mp.o_parts = o_parts;
+  mp.lse_parts = lse_parts;
+  mp.P = P;
+  mp.R = R;
+  mp.o_out = o_out;
+  mp.o_f32 = o_dtype == ATTN_F32;
+  mp.lse_out = lse_out;
+  mp.accumulate = accumulate ? 1 : 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 128) merge_lse_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(mp);
+  else merge_lse_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(mp);
+  ATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+attn_status_t attn_device_status(int reset, int* site) {
+  uint32_t v = 0;
+  ATTN_CUDA(cudaDeviceSynchronize());
+  ATTN_CUDA(cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(v)));
+  if (reset) {
+    const uint32_t z = 0;
+    ATTN_CUDA(cudaMemcpyToSymbol(g_dev_status, &z, sizeof(z)));
+  }
+  if (site) *site = (int)(v & 0xFFFFu);
+  if (v == 0) return ATTN_OK;
+  return ((v >> 16) == ATTN_DEV_TIMEOUT) ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_set_wait_limit_ns(unsigned long long ns) {
+  if (ns == 0) return ATTN_ERR_INVALID_ARG;
+  const uint64_t v = ns;
+  ATTN_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+  return ATTN_OK;
+}
+
+attn_status_t attn_debug_wait_probe(unsigned long long limit_ns) {
+  if (limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000) return ATTN_ERR_INVALID_ARG;
+  uint64_t old = 0;
+  ATTN_CUDA(cudaMemcpyFromSymbol(&old, g_wait_limit_ns, sizeof(old)));
+  const uint64_t v = limit_ns;
+  ATTN_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+  wait_probe_kernel<<<1, 32>>>();
+  const cudaError_t e1 = cudaGetLastError();
+  const cudaError_t e2 = cudaDeviceSynchronize();
+  ATTN_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &old, sizeof(old)));
+  if (e1 != cudaSuccess) return cuda_fail(e1);
+  if (e2 != cudaSuccess) return cuda_fail(e2);
+  return attn_device_status(0, nullptr);
+}
+
+}  // extern "C"

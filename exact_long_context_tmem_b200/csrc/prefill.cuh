@@ -1,0 +1,388 @@
+// Exact GQA prefill on tcgen05: one CTA computes two 128-row query tiles ("slots") that
+// share every K/V tile, so each K/V byte staged in shared memory feeds 256 query rows.
+//
+// Method (ONNX Runtime CPU GQA analysis, "Flash Attention tiling"): for each key block
+// compute the score block, update the running row max and row sum (online softmax), and
+// accumulate P.V into the output; the S x T score matrix never leaves the SM.
+//
+// Roles (384 threads):
+//   warp 0        TMA producer: Q tiles once, then K_j / V_j through an NST-stage ring
+//   warp 1        TMEM allocator; lane 0 issues every tcgen05.mma and commit
+//   warps 4..7    softmax + epilogue for slot 0 (one thread per TMEM lane = query row)
+//   warps 8..11   softmax + epilogue for slot 1
+// TMEM columns: S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// P (bf16, two per column) overwrites the first 64 columns of its S region.  MMA order per
+// key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1) — so S_s(j+1) completing implies PV_s(j)
+// completed, and the softmax warps may rescale O_s and overwrite P_s in place.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace attn {
+
+struct PrefillParams {
+  int B, Hq, Hkv, D, S, T, G;
+  int causal;
+  long long q_pos0, kv_pos0;
+  float scale_log2;  // scale * log2(e)
+  int n_qtiles;      // ceil(S / 128)
+  int pair_heads;    // 1: the slots are heads 2u, 2u+1 of one KV group at one query tile
+  int n_head_units;  // Hq/2 (paired heads) or Hq
+  int n_q_units;     // n_qtiles (paired heads) or ceil(n_qtiles / 2)
+  int n_items;       // B * n_head_units * n_q_units
+  void* o;
+  int o_f32;
+  float* lse;
+};
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int BM = 128;                 // query rows per slot
+  static constexpr int BN = 128;                 // keys per tile
+  static constexpr int NST = (D == 128) ? 2 : 3;  // K/V ring stages
+  static constexpr int BOX_BYTES = 128 * 128;     // one TMA box: 128 rows x 64 bf16
+  static constexpr int NBOX = D / 64;             // boxes per tile along D
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + NST * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NST * TILE_BYTES;
+  static constexpr int N_BARS = 1 + 4 * NST + 2 + 2 + 1 + 1;
+  static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when max grows > 2^8
+};
+
+struct PrefillItem {
+  int b, head[2], q_lo[2];
+  bool active[2];
+  int n_tiles;
+  int kvh;
+};
+
+__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int idx) {
+  PrefillItem it;
+  const int per_q = p.B * p.n_head_units;
+  const int qunit = p.n_q_units - 1 - idx / per_q;  // heaviest causal tiles first
+  const int rem = idx % per_q;
+  it.b = rem / p.n_head_units;
+  const int hunit = rem % p.n_head_units;
+  for (int s = 0; s < 2; ++s) {
+    int head, qt;
+    if (p.pair_heads) {
+      head = 2 * hunit + s;
+      qt = qunit;
+    } else {
+      head = hunit;
+      qt = 2 * qunit + s;
+    }
+    it.head[s] = head;
+    it.q_lo[s] = qt * 128;
+    it.active[s] = it.q_lo[s] < p.S;
+  }
+  it.kvh = it.head[0] / p.G;
+  int n = 0;
+  for (int s = 0; s < 2; ++s) {
+    if (!it.active[s]) continue;
+    long long kv_end = p.T;
+    if (p.causal) {
+      const long long q_last = (long long)min(p.S, it.q_lo[s] + 128) - 1;
+      long long e = p.q_pos0 + q_last - p.kv_pos0 + 1;
+      kv_end = e < kv_end ? e : kv_end;
+    }
+    if (kv_end < 0) kv_end = 0;
+    const int ns = (int)((kv_end + 127) / 128);
+    n = ns > n ? ns : n;
+  }
+  it.n_tiles = n;
+  return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  using C = PrefillCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + C::NST;
+  uint64_t* v_full = k_empty + C::NST;
+  uint64_t* v_empty = v_full + C::NST;
+  uint64_t* s_full = v_empty + C::NST;  // [2]
+  uint64_t* p_full = s_full + 2;        // [2]
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain = o_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const PrefillItem it = prefill_item(p, blockIdx.x);
+  const int n = it.n_tiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < C::NST; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      uint8_t* sQ = smem + C::OFF_Q;
+      mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+      for (int s = 0; s < 2; ++s)
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(sQ + s * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, q_full, bx * 64, it.head[s], it.q_lo[s],
+                      it.b);
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j % C::NST;
+        const uint32_t ph = (j / C::NST) & 1;
+        if (!mbar_wait(&k_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; break; }
+        mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem + C::OFF_K + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmK, &k_full[st], bx * 64, it.kvh,
+                      j * 128, it.b);
+        if (!mbar_wait(&v_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; issued = 2 * j + 1; break; }
+        mbar_arrive_expect_tx(&v_full[st], C::TILE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem + C::OFF_V + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmV, &v_full[st], bx * 64, it.kvh,
+                      j * 128, it.b);
+        issued = 2 * j + 2;
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA's shared memory is released.
+        mbar_wait_drain(q_full, 0, SITE_PF_DRAIN);
+        const int nk = (issued + 1) / 2, nv = issued / 2;
+        for (int j = (nk > C::NST ? nk - C::NST : 0); j < nk; ++j)
+          mbar_wait_drain(&k_full[j % C::NST], (j / C::NST) & 1, SITE_PF_DRAIN);
+        for (int j = (nv > C::NST ? nv - C::NST : 0); j < nv; ++j)
+          mbar_wait_drain(&v_full[j % C::NST], (j / C::NST) & 1, SITE_PF_DRAIN);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc_f16(128, 128, false, false, true);
+      constexpr uint32_t idesc_pv = make_idesc_f16(128, D, false, true, true);
+      const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+      const uint32_t sK = smem_u32(smem + C::OFF_K);
+      const uint32_t sV = smem_u32(smem + C::OFF_V);
+      const uint32_t tS[2] = {tmem + 0, tmem + 128};
+      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      auto issue_qk = [&](int s, int st) {
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+          const uint64_t da = make_sdesc_sw128(sQ + s * C::TILE_BYTES + off, 16, 1024);
+          const uint64_t db = make_sdesc_sw128(sK + st * C::TILE_BYTES + off, 16, 1024);
+          mma_ss(tS[s], da, db, idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int s, int st, bool acc) {
+        for (int kk = 0; kk < 128 / 16; ++kk) {
+          const uint64_t db = make_sdesc_sw128(sV + st * C::TILE_BYTES + kk * 16 * 128, C::BOX_BYTES, 1024);
+          mma_ts(tO[s], tS[s] + kk * 8, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_full, 0, SITE_PF_MMA_Q);
+      if (ok && n > 0) {
+        ok = mbar_wait(&k_full[0], 0, SITE_PF_MMA_K);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          mma_commit(&s_full[0]);
+          issue_qk(1, 0);
+          mma_commit(&s_full[1]);
+          mma_commit(&k_empty[0]);
+        }
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j % C::NST;
+        const uint32_t ph = (j / C::NST) & 1;
+        const bool more = j + 1 < n;
+        const int st1 = (j + 1) % C::NST;
+        const uint32_t ph1 = ((j + 1) / C::NST) & 1;
+        if (!(ok = mbar_wait(&v_full[st], ph, SITE_PF_MMA_V))) break;
+        if (!(ok = mbar_wait(&p_full[0], j & 1, SITE_PF_MMA_P))) break;
+        tc_fence_after();
+        issue_pv(0, st, j > 0);
+        if (more) {
+          if (!(ok = mbar_wait(&k_full[st1], ph1, SITE_PF_MMA_K))) break;
+          tc_fence_after();
+          issue_qk(0, st1);
+          mma_commit(&s_full[0]);
+        }
+        if (!(ok = mbar_wait(&p_full[1], j & 1, SITE_PF_MMA_P))) break;
+        tc_fence_after();
+        issue_pv(1, st, j > 0);
+        mma_commit(&v_empty[st]);
+        if (more) {
+          issue_qk(1, st1);
+          mma_commit(&s_full[1]);
+          mma_commit(&k_empty[st1]);
+        }
+      }
+      if (ok && n > 0) mma_commit(o_full);
+      // Drain: every MMA issued above completes before TMEM is released.
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, SITE_PF_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int slot = (warp - 4) >> 2;
+    const int wq = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + slot * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + slot * D + lane_off;
+    const int q_lo = it.q_lo[slot];
+    const long long rel = p.q_pos0 + q_lo + r - p.kv_pos0;  // key index limit (inclusive) for causal
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (!(ok = mbar_wait(&s_full[slot], j & 1, SITE_PF_SM_S))) break;
+      tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_wait_ld();
+      const int kv0 = j * 128;
+      long long lim64 = (long long)p.T - kv0;  // valid iff column < lim
+      if (p.causal) {
+        const long long c2 = rel + 1 - kv0;
+        lim64 = c2 < lim64 ? c2 : lim64;
+      }
+      const int lim = lim64 < 0 ? 0 : (lim64 > 128 ? 128 : (int)lim64);
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      if (lim < 128) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= lim) sr[i] = __float_as_uint(-INFINITY);
+      }
+#pragma unroll
+      for (int i = 0; i < 128; i += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[i]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[i + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(sr[i + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(sr[i + 3]));
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+      const float m_new = fmaxf(m_used, m_tile);
+      if (m_new > m_used + C::RESCALE_THRESHOLD) {
+        const float alpha = ex2_approx(m_used - m_new);  // 0 when m_used = -inf
+        l *= alpha;
+        if (j > 0) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orow[32];
+            tmem_ld32(tO + c * 32, orow);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+            tmem_st32(tO + c * 32, orow);
+          }
+          tmem_wait_st();
+        }
+        m_used = m_new;
+      }
+      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+      float l0 = 0.f, l1 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[i]), p.scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[i + 1]), p.scale_log2, neg_m));
+        l0 += p0;
+        l1 += p1;
+        pk[i >> 1] = pack_bf16x2(p0, p1);
+      }
+      l += l0 + l1;
+      tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[slot]);
+    }
+    // ---- epilogue: O / l -> global, LSE = ln2 * (m + log2 l)
+    const int row = q_lo + r;
+    const bool row_ok = it.active[slot] && row < p.S;
+    const bool have_o = n > 0;
+    if (ok && have_o) {
+      ok = mbar_wait(o_full, 0, SITE_PF_EPI_O);
+      tc_fence_after();
+    }
+    if (ok && row_ok) {
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const long long orow = (((long long)it.b * p.S + row) * p.Hq + it.head[slot]) * D;
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        if (have_o) {
+          tmem_ld32(tO + c * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (p.o_f32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]) * inv_l, __uint_as_float(v[4 * i + 1]) * inv_l,
+                                 __uint_as_float(v[4 * i + 2]) * inv_l, __uint_as_float(v[4 * i + 3]) * inv_l);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) + orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]) * inv_l, __uint_as_float(v[8 * i + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l, __uint_as_float(v[8 * i + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l, __uint_as_float(v[8 * i + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l, __uint_as_float(v[8 * i + 7]) * inv_l);
+            dst[i] = w;
+          }
+        }
+      }
+      if (p.lse) {
+        const float lse = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        p.lse[((long long)it.b * p.S + row) * p.Hq + it.head[slot]] = lse;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

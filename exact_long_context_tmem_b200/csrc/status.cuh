@@ -1,0 +1,49 @@
+// Device-side status word and wait limit shared by every kernel of the library.
+// The library is one CUDA translation unit, so these globals exist once per device.
+#pragma once
+
+#include <cstdint>
+
+namespace attn {
+
+enum DeviceErrorCode : uint32_t {
+  ATTN_DEV_OK = 0,
+  ATTN_DEV_TIMEOUT = 1,  // a bounded wait ran out
+};
+
+// Wait sites, recorded with the error so a timeout names the wait that gave up.
+enum WaitSite : int {
+  SITE_PROBE = 1,
+  SITE_PF_LOAD_EMPTY = 10,
+  SITE_PF_MMA_Q = 11,
+  SITE_PF_MMA_K = 12,
+  SITE_PF_MMA_V = 13,
+  SITE_PF_MMA_P = 14,
+  SITE_PF_SM_S = 15,
+  SITE_PF_EPI_O = 16,
+  SITE_PF_DRAIN = 17,
+  SITE_DC_LOAD_EMPTY = 30,
+  SITE_DC_MMA_K = 31,
+  SITE_DC_MMA_V = 32,
+  SITE_DC_MMA_P = 33,
+  SITE_DC_SM_S = 34,
+  SITE_DC_SM_O = 35,
+  SITE_DC_SM_V = 36,
+  SITE_DC_DRAIN = 37,
+  SITE_DC_SM_K = 38,
+};
+
+// (code << 16) | site of the first error since the last reset; 0 when clean.
+__device__ uint32_t g_dev_status = 0;
+// Upper bound for any single mbarrier wait, in nanoseconds of %globaltimer.
+__device__ uint64_t g_wait_limit_ns = 2000000000ull;
+
+__device__ __forceinline__ void record_device_error(uint32_t code, int site) {
+  atomicCAS(&g_dev_status, 0u, (code << 16) | (uint32_t)(site & 0xFFFF));
+}
+
+__device__ __forceinline__ bool device_error_set() {
+  return *reinterpret_cast<volatile uint32_t*>(&g_dev_status) != 0u;
+}
+
+}  // namespace attn

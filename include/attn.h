@@ -1,0 +1,208 @@
+/*
+ * attn.h — C ABI of libattn.so: exact long-context attention on NVIDIA B200 (sm_100a).
+ *
+ * The library computes exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T + causal mask) V
+ * with grouped-query heads, tile by tile with an online softmax so the S x T score
+ * matrix never exists in memory; decode splits the key range into partials that a
+ * log-sum-exp reduce merges exactly; a host streamer feeds (query block, key chunk)
+ * sub-tasks from pinned host memory under a device-memory budget and merges their
+ * partials the same way.
+ *
+ * Sources for the operations (web pages; titles and sections):
+ *   [CQSA]  "Stream-CQSA: avoiding out-of-memory in attention computation through flexible
+ *           workload scheduling" (euno.news summary of arXiv 2604.20819), Methodology 1-4,
+ *           Results.
+ *   [COOPT] "LLM-CoOpt: a co-design and optimization framework for efficient LLM inference on
+ *           heterogeneous platforms" (euno.news summary of arXiv 2602.09323), Methodology 1-3.
+ *   [ORT-CPU] "ONNX Runtime CPU GQA optimization: Flash Attention and Flash Decoding"
+ *           (analysis of onnxruntime PR 28695), Code analysis 1-2, Reviewer feedback.
+ *   [ORT-QSA] "ONNX Runtime CUDA packed sparse attention optimization" (analysis of
+ *           onnxruntime PR 33328), Code analysis 1.
+ *
+ * Conventions for every entry point
+ *   - Device pointers are plain CUDA device addresses owned by the caller; the library never
+ *     frees or keeps them.  Host pointers are used only during the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Device
+ *     calls enqueue work and return without synchronising, except attn_chunked_stream, which
+ *     returns after its last device-to-host copy has completed.
+ *   - Every argument is validated before any CUDA call; an invalid call returns an error
+ *     status, launches nothing and never aborts or prints.
+ *   - Layouts are row-major.  Q and O are token-major [B, S, Hq, D]; K and V are
+ *     [B, T, Hkv, D]; the row log-sum-exp LSE is float32 [B, S, Hq] (same row order as O),
+ *     natural log, including the score scale.  Query head h reads KV head h / (Hq / Hkv).
+ *   - Supported: D in {64, 128}; bf16 Q/K/V; FP8 E4M3 K/V (decode); Hq % Hkv == 0;
+ *     Hq / Hkv <= 16 for decode.  All base pointers 16-byte aligned.
+ *   - Thread safety: calls may be made from several host threads at once.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or combination */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels implement (e.g. D=96) */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed; see attn_last_cuda_error() */
+  ATTN_ERR_BUDGET = 4,      /* the streamer's smallest plan does not fit the device budget */
+  ATTN_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (device status word) */
+  ATTN_ERR_INJECTED = 6     /* a host-side injected failure (tests of the error paths) */
+} attn_status_t;
+
+typedef enum { ATTN_BF16 = 0, ATTN_FP8_E4M3 = 1, ATTN_F32 = 2 } attn_dtype_t;
+
+typedef struct {
+  int B;       /* batch */
+  int Hq;      /* query heads */
+  int Hkv;     /* key/value heads; Hq % Hkv == 0 ([COOPT] Opt-GQA: heads share K/V in groups) */
+  int D;       /* head dimension, 64 or 128 */
+  float scale; /* score scale > 0, normally 1/sqrt(D) */
+} attn_dims_t;
+
+/* ------------------------------------------------------------------------------------------
+ * attn_prefill — exact (optionally causal) GQA attention of S query rows over T keys.
+ *
+ * Follows [ORT-CPU] Code analysis 1 (tiled computation: per key block, score block, online
+ * softmax running max and sum, fused P·V accumulation) on tcgen05 tensor cores, with the
+ * definition of [CQSA] Methodology 2.  Query row i sits at absolute position q_pos0 + i, key j
+ * at kv_pos0 + j ([ORT-QSA] Code analysis 1: position = past length + local index); with
+ * causal != 0 row i sees key j iff kv_pos0 + j <= q_pos0 + i.  Tiles wholly above the
+ * diagonal or past T are never computed.
+ *
+ *   q    device bf16 [B, S, Hq, D]     k, v  device bf16 [B, T, Hkv, D]
+ *   o    device [B, S, Hq, D], bf16 (o_dtype = ATTN_BF16) or float32 (ATTN_F32)
+ *   lse  device float32 [B, S, Hq] or NULL.  Rows that see no key get O = 0, LSE = -inf.
+ *   S, T >= 0 (S = 0 or B = 0 is a no-op); q_pos0, kv_pos0 >= 0.
+ * Returns ATTN_OK after enqueueing on `stream`.
+ * ------------------------------------------------------------------------------------------ */
+ATTN_API attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o, attn_dtype_t o_dtype,
+                           float* lse, attn_dims_t dims, int S, int T, int causal, long long q_pos0,
+                           long long kv_pos0, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * attn_decode_splitkv — one query token per sequence over a ragged KV cache.
+ *
+ * Flash Decoding ([ORT-CPU] Code analysis 2): the key range of each (sequence, KV head) is cut
+ * into num_splits chunks, each producing a partial softmax state, and a log-sum-exp reduce
+ * merges them.  Sequence b's query sits at position kv_lens[b] - 1 and sees keys
+ * [0, kv_lens[b]).  Lengths stay on the device (no host read-back).  Cache slots at or past
+ * kv_lens[b] are never used, whatever they hold (NaN included).  kv_lens[b] == 0 gives O = 0,
+ * LSE = -inf.
+ *
+ *   q        device bf16 [B, Hq, D]
+ *   k, v     device [B, Tmax, Hkv, D]: bf16 (kv_dtype = ATTN_BF16) or E4M3 codes (ATTN_FP8_E4M3)
+ *   k_scale, v_scale  device float32 [B, Tmax, Hkv] dequantisation multipliers for FP8
+ *            ([COOPT] Opt-KV FP8 cache); must be NULL for bf16.  Dequantised value = code * scale.
+ *   kv_lens  device int32 [B], each in [0, Tmax]
+ *   num_splits  0 = automatic (fills the GPU), else 1..4096
+ *   o        device bf16 [B, Hq, D];  lse  device float32 [B, Hq] or NULL
+ *   ws       device workspace of at least attn_decode_workspace_bytes(dims, Tmax, num_splits)
+ *            bytes, owned by the caller; may be NULL when that size is 0.
+ * ------------------------------------------------------------------------------------------ */
+ATTN_API size_t attn_decode_workspace_bytes(attn_dims_t dims, int Tmax, int num_splits);
+ATTN_API int attn_decode_num_splits(attn_dims_t dims, int Tmax, int num_splits); /* the split count used */
+ATTN_API attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                  const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax,
+                                  attn_dims_t dims, int num_splits, void* o, float* lse, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * attn_merge_lse — exact log-sum-exp merge of P partial results per row.
+ *
+ * [ORT-CPU] Code analysis 2 (the reduce phase that merges per-chunk partial softmax states by
+ * log-sum-exp) and [CQSA] Methodology 2-3 (sub-results recombine to the full result):
+ * lse = log sum_p exp(lse_p),
+ * o = sum_p exp(lse_p - lse) o_p; parts with lse_p = -inf add nothing; a row with every part
+ * empty gets o = 0, lse = -inf.
+ *
+ *   o_parts   device float32 [P, R, D];  lse_parts device float32 [P, R]
+ *   o_out     device [R, D], bf16 or float32 (o_dtype);  lse_out device float32 [R] or NULL
+ *   accumulate != 0: (o_out, lse_out) already hold a partial (o_out float32, lse_out non-NULL)
+ *             that is merged in place with the P parts.
+ *   P >= 1 (P = 0 valid only with accumulate), R >= 0, D in {64, 128}.
+ * ------------------------------------------------------------------------------------------ */
+ATTN_API attn_status_t attn_merge_lse(const float* o_parts, const float* lse_parts, int P, long long R, int D,
+                             void* o_out, attn_dtype_t o_dtype, float* lse_out, int accumulate, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Streamer: exact causal (or full) self-attention over S tokens whose Q, K, V, O, LSE live in
+ * host memory, computed under a device-memory budget.
+ *
+ * [CQSA] Methodology 2-4: attention is split into independent sub-tasks — here (query block,
+ * key chunk) rectangles that cover every visible (query, key) pair exactly once — queued and
+ * streamed host->device on a copy stream, computed on the compute stream, and recombined by
+ * the log-sum-exp merge; finished blocks are swapped back to host memory.  A controller picks
+ * the block sizes from the budget ([CQSA] Methodology 4; its Limitations section calls the
+ * block-size rule a plain heuristic).
+ *
+ *   q_h, k_h, v_h  host bf16 [B, S, Hq, D] / [B, S, Hkv, D]; pinned memory lets copies overlap
+ *   o_h            host bf16 [B, S, Hq, D];  lse_h host float32 [B, S, Hq] or NULL
+ *   chunk_tokens   key chunk length (0 = the controller picks); multiple of 128
+ *   device_budget_bytes  upper bound on every device allocation the call makes
+ *   compute_stream, copy_stream: cudaStream_t or NULL (the call then creates its own)
+ *   stats          optional out-parameter
+ * Allocates device buffers (counted against the budget) and frees them before returning.
+ * Returns ATTN_ERR_BUDGET, without allocating, if the smallest plan does not fit.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct {
+  long long q_block;      /* query rows per block */
+  long long kv_chunk;     /* keys per chunk */
+  long long n_tasks;      /* (query block, key chunk) sub-tasks */
+  long long device_bytes; /* bytes the plan allocates on the device */
+} attn_stream_plan_t;
+
+typedef struct {
+  attn_stream_plan_t plan;
+  long long h2d_bytes;     /* host->device bytes copied */
+  long long d2h_bytes;     /* device->host bytes copied */
+  double ms_total;         /* wall time of the call (host clock) */
+  double ms_compute;       /* summed device time of prefill + merge launches (CUDA events) */
+} attn_stream_stats_t;
+
+ATTN_API attn_status_t attn_stream_plan(attn_dims_t dims, long long S, int causal, long long chunk_tokens,
+                               size_t device_budget_bytes, attn_stream_plan_t* plan);
+/* The idx-th task of a plan in execution order: first query row and first key of its rectangle. */
+ATTN_API attn_status_t attn_stream_task(const attn_stream_plan_t* plan, long long S, int causal, long long idx,
+                               long long* q_start, long long* kv_start);
+ATTN_API attn_status_t attn_chunked_stream(const void* q_h, const void* k_h, const void* v_h, void* o_h, float* lse_h,
+                                  attn_dims_t dims, long long S, int causal, long long chunk_tokens,
+                                  size_t device_budget_bytes, void* compute_stream, void* copy_stream,
+                                  attn_stream_stats_t* stats);
+
+/* ------------------------------------------------------------------------------------------
+ * Status and diagnostics
+ * ------------------------------------------------------------------------------------------ */
+ATTN_API const char* attn_status_string(attn_status_t status);
+/* Last CUDA error code seen by this host thread inside the library (0 = none). */
+ATTN_API int attn_last_cuda_error(void);
+/* Reads the device status word of the current device (synchronises the device).  Returns
+ * ATTN_ERR_TIMEOUT if a kernel's bounded wait ran out since the last reset, and stores the
+ * wait site in *site when site != NULL.  reset != 0 clears the word. */
+ATTN_API attn_status_t attn_device_status(int reset, int* site);
+/* Upper bound of any single in-kernel wait, in nanoseconds (default 2e9). */
+ATTN_API attn_status_t attn_set_wait_limit_ns(unsigned long long ns);
+/* Launches one tiny kernel that waits on an mbarrier nothing ever arrives at, with the given
+ * limit; the wait runs out, the kernel records ATTN_ERR_TIMEOUT and returns.  Used to test
+ * the timeout path without faulting or hanging the GPU.  Synchronises the device. */
+ATTN_API attn_status_t attn_debug_wait_probe(unsigned long long limit_ns);
+/* Host-side fault injection for the streamer: the nth (1-based) host->device copy (what = 1)
+ * or device allocation (what = 2) of the next attn_chunked_stream call fails with
+ * ATTN_ERR_INJECTED.  what = 0 disarms. */
+ATTN_API attn_status_t attn_debug_inject(int what, long long nth);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ATTN_H_ */
