@@ -378,6 +378,15 @@ attn_status_t attn_set_wait_limit_ns(unsigned long long ns) {
   return ATTN_OK;
 }
 
+#ifdef ATTN_TRACE
+// Trace builds only: point the progress trace at host-mapped memory (device address).
+ATTN_API attn_status_t attn_debug_set_trace(void* dev_ptr) {
+  uint32_t* p = static_cast<uint32_t*>(dev_ptr);
+  ATTN_CUDA(cudaMemcpyToSymbol(g_trace, &p, sizeof(p)));
+  return ATTN_OK;
+}
+#endif
+
 attn_status_t attn_debug_wait_probe(unsigned long long limit_ns) {
   if (limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000) return ATTN_ERR_INVALID_ARG;
   uint64_t old = 0;

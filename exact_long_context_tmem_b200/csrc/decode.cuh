@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     const long long kv_row0 = (long long)b * p.Tmax;
     if (FP8) {  // convert K_0
-      ok = mbar_wait(&k_full[0], 0, SITE_DC_SM_K);
+      ok = mbar_wait_warp(&k_full[0], 0, SITE_DC_SM_K);
       if (ok) {
         convert_row_e4m3(smem + C::OFF_K, smem + C::OFF_KC, t, t0 + t < t1);
         mbar_arrive(&k_empty[0]);
@@ -340,7 +340,8 @@ __global__ void __launch_bounds__(192, 1)
         ks = p.k_scale[(kv_row0 + tok) * p.Hkv + kvh];
         vs = p.v_scale[(kv_row0 + tok) * p.Hkv + kvh];
       }
-      if (!(ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
+      // tcgen05.ld/st are warp-collective: every lane takes the same branch around them.
+      if (!(ok = mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
       tc_fence_after();
       uint32_t sv[16];
       tmem_ld16(tS0 + (j & 1) * 16 + lane_off, sv);
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       mbar_arrive(&red_bar[j & 1]);
-      if (!(ok = mbar_wait(&red_bar[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
+      if (!(ok = mbar_wait_warp(&red_bar[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
       bool need = false;
       float alpha[16];
 #pragma unroll
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       if (need && j > 0) {  // rescale O^T row t (element d = t of every query row)
-        if (!(ok = mbar_wait(o_ready, (j - 1) & 1, SITE_DC_SM_O))) break;
+        if (!(ok = mbar_wait_warp(o_ready, (j - 1) & 1, SITE_DC_SM_O))) break;
         tc_fence_after();
         uint32_t orow[16];
         tmem_ld16(tO + lane_off, orow);
@@ -402,14 +403,14 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (FP8) {
         // V_j codes -> f16 (needs PV(j-1) finished reading the converted V tile)
-        if (j > 0 && !(ok = mbar_wait(o_ready, (j - 1) & 1, SITE_DC_SM_O))) break;
-        if (!(ok = mbar_wait(&v_full[st], ph, SITE_DC_SM_V))) break;
+        if (j > 0 && !(ok = mbar_wait_warp(o_ready, (j - 1) & 1, SITE_DC_SM_O))) break;
+        if (!(ok = mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V))) break;
         convert_row_e4m3(smem + C::OFF_V + st * C::KV_TILE, smem + C::OFF_VC, t, valid);
         mbar_arrive(&v_empty[st]);
       } else if (t1 - (t0 + j * 128) < 128) {
         // last, partial tile: cache slots past the length may hold anything (NaN included);
         // zero those V rows so 0-probability x slot cannot poison the sum.
-        if (!(ok = mbar_wait(&v_full[st], ph, SITE_DC_SM_V))) break;
+        if (!(ok = mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V))) break;
         if (!valid) {
           uint4* r0 = reinterpret_cast<uint4*>(smem + C::OFF_V + st * C::KV_TILE + t * 128);
           uint4* r1 = reinterpret_cast<uint4*>(smem + C::OFF_V + st * C::KV_TILE + 128 * 128 + t * 128);
@@ -422,7 +423,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(&p_full[j & 1]);
       if (FP8 && j + 1 < n) {  // K_{j+1} codes -> f16 (S(j) has finished reading the converted K tile)
         const int st1 = (j + 1) % C::NST;
-        if (!(ok = mbar_wait(&k_full[st1], ((j + 1) / C::NST) & 1, SITE_DC_SM_K))) break;
+        if (!(ok = mbar_wait_warp(&k_full[st1], ((j + 1) / C::NST) & 1, SITE_DC_SM_K))) break;
         convert_row_e4m3(smem + C::OFF_K + st1 * C::KV_TILE, smem + C::OFF_KC, t, tok + 128 < t1);
         mbar_arrive(&k_empty[st1]);
         fence_proxy_async_smem();
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       mbar_arrive(sum_bar);
-      ok = mbar_wait(sum_bar, 0, SITE_DC_SM_S) && mbar_wait(o_ready, (n - 1) & 1, SITE_DC_SM_O);
+      ok = mbar_wait_warp(sum_bar, 0, SITE_DC_SM_S) && mbar_wait_warp(o_ready, (n - 1) & 1, SITE_DC_SM_O);
     }
     if (ok) {
       tc_fence_after();

@@ -140,13 +140,16 @@ __global__ void __launch_bounds__(384, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
+    if (lane == 0) ATTN_TRACE_AT(1, 1, 0);
     tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
+    if (lane == 0) ATTN_TRACE_AT(1, 2, 0);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  if (threadIdx.x == 0) ATTN_TRACE_AT(0, 3, n);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -165,11 +168,13 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < n && ok; ++j) {
         const int st = j % C::NST;
         const uint32_t ph = (j / C::NST) & 1;
+        ATTN_TRACE_AT(0, 4, j);
         if (!mbar_wait(&k_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; break; }
         mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem + C::OFF_K + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmK, &k_full[st], bx * 64, it.kvh,
                       j * 128, it.b);
+        ATTN_TRACE_AT(0, 5, j);
         if (!mbar_wait(&v_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; issued = 2 * j + 1; break; }
         mbar_arrive_expect_tx(&v_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
@@ -177,6 +182,7 @@ __global__ void __launch_bounds__(384, 1)
                       j * 128, it.b);
         issued = 2 * j + 2;
       }
+      ATTN_TRACE_AT(0, 6, issued);
       if (!ok) {
         // Let every copy already issued land before the CTA's shared memory is released.
         mbar_wait_drain(q_full, 0, SITE_PF_DRAIN);
@@ -212,7 +218,9 @@ __global__ void __launch_bounds__(384, 1)
           mma_ts(tO[s], tS[s] + kk * 8, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
+      ATTN_TRACE_AT(1, 3, 0);
       bool ok = mbar_wait(q_full, 0, SITE_PF_MMA_Q);
+      ATTN_TRACE_AT(1, 4, ok);
       if (ok && n > 0) {
         ok = mbar_wait(&k_full[0], 0, SITE_PF_MMA_K);
         if (ok) {
@@ -230,8 +238,11 @@ __global__ void __launch_bounds__(384, 1)
         const bool more = j + 1 < n;
         const int st1 = (j + 1) % C::NST;
         const uint32_t ph1 = ((j + 1) / C::NST) & 1;
+        ATTN_TRACE_AT(1, 5, j);
         if (!(ok = mbar_wait(&v_full[st], ph, SITE_PF_MMA_V))) break;
+        ATTN_TRACE_AT(1, 6, j);
         if (!(ok = mbar_wait(&p_full[0], j & 1, SITE_PF_MMA_P))) break;
+        ATTN_TRACE_AT(1, 7, j);
         tc_fence_after();
         issue_pv(0, st, j > 0);
         if (more) {
@@ -240,7 +251,9 @@ __global__ void __launch_bounds__(384, 1)
           issue_qk(0, st1);
           mma_commit(&s_full[0]);
         }
+        ATTN_TRACE_AT(1, 8, j);
         if (!(ok = mbar_wait(&p_full[1], j & 1, SITE_PF_MMA_P))) break;
+        ATTN_TRACE_AT(1, 9, j);
         tc_fence_after();
         issue_pv(1, st, j > 0);
         mma_commit(&v_empty[st]);
@@ -251,9 +264,11 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       if (ok && n > 0) mma_commit(o_full);
+      ATTN_TRACE_AT(1, 10, ok);
       // Drain: every MMA issued above completes before TMEM is released.
       mma_commit(drain);
-      mbar_wait_drain(drain, 0, SITE_PF_DRAIN);
+      const bool drained = mbar_wait_drain(drain, 0, SITE_PF_DRAIN);
+      ATTN_TRACE_AT(1, 11, drained);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -269,7 +284,10 @@ __global__ void __launch_bounds__(384, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      if (!(ok = mbar_wait(&s_full[slot], j & 1, SITE_PF_SM_S))) break;
+      if (r == 0) ATTN_TRACE_AT(2 + slot, 1, j);
+      // tcgen05.ld/st are warp-collective: every lane takes the same branch around them.
+      if (!(ok = mbar_wait_warp(&s_full[slot], j & 1, SITE_PF_SM_S))) break;
+      if (r == 0) ATTN_TRACE_AT(2 + slot, 2, j);
       tc_fence_after();
       uint32_t sr[128];
 #pragma unroll
@@ -297,10 +315,14 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
       const float m_new = fmaxf(m_used, m_tile);
-      if (m_new > m_used + C::RESCALE_THRESHOLD) {
-        const float alpha = ex2_approx(m_used - m_new);  // 0 when m_used = -inf
-        l *= alpha;
-        if (j > 0) {
+      const bool need = m_new > m_used + C::RESCALE_THRESHOLD;
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2_approx(m_used - m_new) : 1.f;  // 0 when m_used = -inf
+        if (need) {
+          l *= alpha;
+          m_used = m_new;
+        }
+        if (j > 0) {  // the whole warp rescales its 32 rows of O (factor 1 where unchanged)
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orow[32];
@@ -312,7 +334,6 @@ __global__ void __launch_bounds__(384, 1)
           }
           tmem_wait_st();
         }
-        m_used = m_new;
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
       float l0 = 0.f, l1 = 0.f;
@@ -326,9 +347,11 @@ __global__ void __launch_bounds__(384, 1)
         pk[i >> 1] = pack_bf16x2(p0, p1);
       }
       l += l0 + l1;
+      if (r == 0) ATTN_TRACE_AT(2 + slot, 3, j);
       tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
+      if (r == 0) ATTN_TRACE_AT(2 + slot, 4, j);
       tc_fence_before();
       mbar_arrive(&p_full[slot]);
     }
@@ -336,22 +359,25 @@ __global__ void __launch_bounds__(384, 1)
     const int row = q_lo + r;
     const bool row_ok = it.active[slot] && row < p.S;
     const bool have_o = n > 0;
+    if (r == 0) ATTN_TRACE_AT(4 + slot, 1, ok);
     if (ok && have_o) {
-      ok = mbar_wait(o_full, 0, SITE_PF_EPI_O);
+      ok = mbar_wait_warp(o_full, 0, SITE_PF_EPI_O);
       tc_fence_after();
     }
-    if (ok && row_ok) {
+    if (r == 0) ATTN_TRACE_AT(4 + slot, 2, ok);
+    if (ok) {
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       const long long orow = (((long long)it.b * p.S + row) * p.Hq + it.head[slot]) * D;
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        if (have_o) {
+        if (have_o) {  // warp-collective load for every lane; only rows < S are stored
           tmem_ld32(tO + c * 32, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;
         }
+        if (!row_ok) continue;
         if (p.o_f32) {
           float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + orow + c * 32);
 #pragma unroll
@@ -371,17 +397,19 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (p.lse) {
+      if (p.lse && row_ok) {
         const float lse = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
         p.lse[((long long)it.b * p.S + row) * p.Hq + it.head[slot]] = lse;
       }
     }
   }
   tc_fence_before();
+  if (threadIdx.x == 0) ATTN_TRACE_AT(6, 1, 0);
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+    if (lane == 0) ATTN_TRACE_AT(6, 2, 0);
   }
 }
 

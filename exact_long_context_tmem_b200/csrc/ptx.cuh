@@ -79,6 +79,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int si
   return mbar_wait_slow(bar, parity, site, false);
 }
 
+// Wait for roles in which all 32 lanes run the same code: the outcome is made warp-uniform, so a
+// timeout never splits a warp in front of a warp-collective tcgen05 instruction.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int site) {
+  const bool ok = mbar_wait(bar, parity, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, site, true);

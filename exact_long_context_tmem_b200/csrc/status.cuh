@@ -46,4 +46,23 @@ __device__ __forceinline__ bool device_error_set() {
   return *reinterpret_cast<volatile uint32_t*>(&g_dev_status) != 0u;
 }
 
+// Optional progress trace for diagnosing a stalled kernel (compiled in only with -DATTN_TRACE):
+// each role writes (stage << 16 | iteration) into host-mapped memory that the host can read
+// while the kernel is still running.
+#ifdef ATTN_TRACE
+__device__ uint32_t* g_trace = nullptr;
+#define ATTN_TRACE_AT(slot, stage, iter)                                                  \
+  do {                                                                                    \
+    volatile uint32_t* t_ = g_trace;                                                      \
+    if (t_) {                                                                             \
+      t_[blockIdx.x * 16 + (slot)] = ((uint32_t)(stage) << 16) | ((uint32_t)(iter) & 0xFFFFu); \
+      __threadfence_system();                                                             \
+    }                                                                                     \
+  } while (0)
+#else
+#define ATTN_TRACE_AT(slot, stage, iter) \
+  do {                                   \
+  } while (0)
+#endif
+
 }  // namespace attn
