@@ -23,6 +23,7 @@ ATTN_BF16, ATTN_FP8_E4M3, ATTN_F32 = 0, 1, 2
 
 EXPORTS = [
     "attn_prefill", "attn_decode_workspace_bytes", "attn_decode_num_splits", "attn_decode_splitkv",
+    "attn_decode_splitkv_noalloc",
     "attn_merge_lse", "attn_stream_plan", "attn_stream_task", "attn_chunked_stream", "attn_status_string",
     "attn_last_cuda_error", "attn_device_status", "attn_set_wait_limit_ns", "attn_debug_wait_probe",
     "attn_debug_inject",
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
     L.attn_decode_num_splits.restype = i
     L.attn_decode_splitkv.argtypes = [vp, vp, vp, i, vp, vp, vp, i, Dims, i, vp, vp, vp, sz, vp]
     L.attn_decode_splitkv.restype = i
+    L.attn_decode_splitkv_noalloc.argtypes = [vp, vp, vp, i, vp, vp, vp, i, Dims, i, vp, vp, vp]
+    L.attn_decode_splitkv_noalloc.restype = i
     L.attn_merge_lse.argtypes = [vp, vp, i, ll, i, vp, i, vp, i, vp]
     L.attn_merge_lse.restype = i
     L.attn_stream_plan.argtypes = [Dims, ll, i, ll, sz, ctypes.POINTER(StreamPlan)]
@@ -170,6 +173,31 @@ def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: 
                                    _ptr(v_scale), _ptr(kv_lens), int(Tmax), dims, int(num_splits), _ptr(o),
                                    _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "attn_decode_splitkv")
+    return o, lse
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def attn_decode_splitkv_noalloc(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: float | None = None,
+                                num_splits: int = 0, o=None, lse=None, want_lse: bool = True, stream=None):
+    """attn_decode_splitkv without a workspace: the split partials live in the library's static
+    device scratch array (see include/attn.h).  For callers that cannot allocate device memory;
+    the outputs o and lse may be passed in preallocated."""
+    _need_cuda(q, k, v, kv_lens, k_scale, v_scale, o, lse)
+    B, Hq, D = q.shape
+    Tmax, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    fp8 = k.dtype in (torch.uint8, torch.float8_e4m3fn)
+    if o is None:
+        o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    st = lib().attn_decode_splitkv_noalloc(_ptr(q), _ptr(k), _ptr(v), ATTN_FP8_E4M3 if fp8 else ATTN_BF16,
+                                           _ptr(k_scale), _ptr(v_scale), _ptr(kv_lens), int(Tmax),
+                                           _dims(B, Hq, Hkv, D, scale), int(num_splits), _ptr(o), _ptr(lse),
+                                           _stream(stream))
+    _check(st, "attn_decode_splitkv_noalloc")
     return o, lse
 
 

@@ -330,6 +330,37 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, a
   return launch_decode<false>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st);
 }
 
+// Split-KV decode without allocation: the split partials live in this static device array
+// (ATTN_NOALLOC_SCRATCH_BYTES per device, held until the process exits).  Host code must not pass
+// the array's name to a kernel — on the host it is only a stand-in — so its device address is
+// looked up once per device with cudaGetSymbolAddress, with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                          const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax,
+                                          attn_dims_t dims, int num_splits, void* o, float* lse, void* stream) {
+  if (!dims_ok(dims) || Tmax < 0 || num_splits < 0 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
+  const size_t need = decode_ws_bytes(dims, decode_splits(dims, Tmax, num_splits));
+  if (need > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_BUDGET;
+  void* ws = nullptr;
+  if (need > 0) {
+    static std::mutex mu;
+    static void* scratch[64] = {};
+    int dev = 0;
+    ATTN_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return ATTN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!scratch[dev]) {
+      void* p = nullptr;
+      ATTN_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+      scratch[dev] = p;
+    }
+    ws = scratch[dev];
+  }
+  return attn_decode_splitkv(q, k, v, kv_dtype, k_scale, v_scale, kv_lens, Tmax, dims, num_splits, o, lse, ws,
+                             need > 0 ? (size_t)ATTN_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+
 attn_status_t attn_merge_lse(const float* o_parts, const float* lse_parts, int P, long long R, int D, void* o_out,
                              attn_dtype_t o_dtype, float* lse_out, int accumulate, void* stream) {
   if (P < 0 || R < 0 || (P == 0 && !accumulate)) return ATTN_ERR_INVALID_ARG;

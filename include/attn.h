@@ -119,6 +119,32 @@ ATTN_API attn_status_t attn_decode_splitkv(const void* q, const void* k, const v
                                   size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * attn_decode_splitkv_noalloc — the same split-KV decode, for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this entry point; it is an integration aid.  Some callers
+ * cannot call cudaMalloc or hand out a workspace: a serving engine that has reserved nearly
+ * all device memory for its own pool, or a latency-critical decode loop in which an allocation
+ * (which may synchronise the device) is not allowed.  This variant takes the same arguments as
+ * attn_decode_splitkv minus the workspace, and keeps the split partials in one static device
+ * array of ATTN_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds until the
+ * process exits.  It allocates nothing.
+ *
+ *   - The first call on a device (with that device current) looks up the array's device
+ *     address; make that first call before any stream capture.
+ *   - Requests whose partials need more than ATTN_NOALLOC_SCRATCH_BYTES
+ *     (attn_decode_workspace_bytes(dims, Tmax, num_splits) > the limit) return ATTN_ERR_BUDGET
+ *     without launching anything; lower num_splits or use attn_decode_splitkv.
+ *   - All calls share the array and it keeps the last call's contents.  Nothing in it needs to
+ *     start at zero (every partial is written before it is read), but calls whose work
+ *     overlaps on the GPU (other streams, other host threads) race on it: serialise them.
+ * ------------------------------------------------------------------------------------------ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (4u << 20)
+ATTN_API attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                          const float* k_scale, const float* v_scale, const int* kv_lens,
+                                          int Tmax, attn_dims_t dims, int num_splits, void* o, float* lse,
+                                          void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * attn_merge_lse — exact log-sum-exp merge of P partial results per row.
  *
  * [ORT-CPU] Code analysis 2 (the reduce phase that merges per-chunk partial softmax states by
