@@ -26,7 +26,7 @@ EXPORTS = [
     "attn_decode_splitkv_noalloc",
     "attn_merge_lse", "attn_stream_plan", "attn_stream_task", "attn_chunked_stream", "attn_status_string",
     "attn_last_cuda_error", "attn_device_status", "attn_set_wait_limit_ns", "attn_debug_wait_probe",
-    "attn_debug_inject",
+    "attn_debug_inject", "attn_debug_exp2",
 ]
 
 
@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
     L.attn_debug_wait_probe.restype = i
     L.attn_debug_inject.argtypes = [i, ll]
     L.attn_debug_inject.restype = i
+    L.attn_debug_exp2.argtypes = [vp, vp, ll, i, vp]
+    L.attn_debug_exp2.restype = i
     _ = f
     _lib = L
     return L
@@ -273,6 +275,15 @@ def attn_debug_wait_probe(limit_ns: int) -> int:
 
 def attn_debug_inject(what: int, nth: int):
     _check(lib().attn_debug_inject(int(what), int(nth)), "attn_debug_inject")
+
+
+def attn_debug_exp2(x, mode: int = 0, stream=None):
+    """Device exp2 of a float32 CUDA tensor: mode 0 = FMA-pipe polynomial, 1 = MUFU ex2.approx."""
+    _need_cuda(x)
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check(lib().attn_debug_exp2(_ptr(x), _ptr(y), x.numel(), int(mode), _stream(stream)), "attn_debug_exp2")
+    return y
 
 
 def attn_status_string(status: int) -> str:

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libattn.so")
 SOURCES = ["api.cu", "stream.cpp"]
-HEADERS = ["ptx.cuh", "status.cuh", "prefill.cuh", "decode.cuh", "merge.cuh"]
+HEADERS = ["ptx.cuh", "status.cuh", "prefill.cuh", "decode.cuh", "decode_fp8.cuh", "merge.cuh"]
 
 
 def nvcc() -> str:

@@ -13,6 +13,7 @@
 
 #include "../../include/attn.h"
 #include "decode.cuh"
+#include "decode_fp8.cuh"
 #include "merge.cuh"
 #include "prefill.cuh"
 
@@ -172,9 +173,11 @@ template <bool FP8>
 static attn_status_t launch_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
                                    const int* kv_lens, int Tmax, const attn_dims_t& d, int P, int split_tokens,
                                    void* o, float* lse, void* ws, cudaStream_t stream) {
-  using C = DecodeCfg<FP8>;
   static std::atomic<uint64_t> smem_done{0};
-  attn_status_t st = ensure_smem(decode_split_sm100<FP8>, C::SMEM_BYTES, smem_done);
+  const int smem_bytes = FP8 ? DecodeFp8Cfg::SMEM_BYTES : DecodeCfg<false>::SMEM_BYTES;
+  const int threads = FP8 ? DecodeFp8Cfg::THREADS : DecodeCfg<false>::THREADS;
+  attn_status_t st = FP8 ? ensure_smem(decode_fp8_sm100, smem_bytes, smem_done)
+                         : ensure_smem(decode_split_sm100<false>, smem_bytes, smem_done);
   if (st != ATTN_OK) return st;
   CUtensorMap mk, mv;
   // With Tmax == 0 every split is empty and no map is read; it still needs a valid base and extent.
@@ -210,7 +213,8 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   dim3 grid(P, d.Hkv, d.B);
-  decode_split_sm100<FP8><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, p);
+  if (FP8) decode_fp8_sm100<<<grid, threads, smem_bytes, stream>>>(mk, mv, p);
+  else decode_split_sm100<false><<<grid, threads, smem_bytes, stream>>>(mk, mv, p);
   ATTN_CUDA(cudaGetLastError());
   if (P > 1) {
     MergeParams mp{};
@@ -230,6 +234,21 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
 }
 
 // ---------------------------------------------------------------- diagnostics
+
+__global__ void exp2_probe_kernel(const float* x, float* y, long long n, int mode) {
+  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 >= n + 1) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  float2 r;
+  if (mode == 0) {
+    r = exp2_poly2(make_float2(a, b));
+  } else {
+    r.x = ex2_approx(a);
+    r.y = ex2_approx(b);
+  }
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
+}
 
 __global__ void wait_probe_kernel() {
   __shared__ uint64_t bar;
@@ -417,6 +436,17 @@ ATTN_API attn_status_t attn_debug_set_trace(void* dev_ptr) {
   return ATTN_OK;
 }
 #endif
+
+attn_status_t attn_debug_exp2(const float* x, float* y, long long n, int mode, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y)) || (mode != 0 && mode != 1)) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  const long long pairs = (n + 1) / 2;
+  const long long blocks = (pairs + 255) / 256;
+  if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  exp2_probe_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
+  ATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
 
 attn_status_t attn_debug_wait_probe(unsigned long long limit_ns) {
   if (limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000) return ATTN_ERR_INVALID_ARG;

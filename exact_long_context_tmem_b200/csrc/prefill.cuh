@@ -289,29 +289,36 @@ __global__ void __launch_bounds__(384, 1)
       if (!(ok = mbar_wait_warp(&s_full[slot], j & 1, SITE_PF_SM_S))) break;
       if (r == 0) ATTN_TRACE_AT(2 + slot, 2, j);
       tc_fence_after();
-      uint32_t sr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-      tmem_wait_ld();
       const int kv0 = j * 128;
-      long long lim64 = (long long)p.T - kv0;  // valid iff column < lim
+      long long lim64 = (long long)p.T - kv0;  // column c is a visible key iff c < lim
       if (p.causal) {
         const long long c2 = rel + 1 - kv0;
         lim64 = c2 < lim64 ? c2 : lim64;
       }
       const int lim = lim64 < 0 ? 0 : (lim64 > 128 ? 128 : (int)lim64);
+      // pass 1: row max over the 128 scores, read from TMEM in two halves
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-      if (lim < 128) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i >= lim) sr[i] = __float_as_uint(-INFINITY);
-      }
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[32], bb[32];
+        tmem_ld32(tS + h * 64, a);
+        tmem_ld32(tS + h * 64 + 32, bb);
+        tmem_wait_ld_regs(a);
+        tmem_wait_ld_regs(bb);
+        if (lim < 128) {
 #pragma unroll
-      for (int i = 0; i < 128; i += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[i]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[i + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(sr[i + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(sr[i + 3]));
+          for (int i = 0; i < 32; ++i) {
+            if (h * 64 + i >= lim) a[i] = __float_as_uint(-INFINITY);
+            if (h * 64 + 32 + i >= lim) bb[i] = __float_as_uint(-INFINITY);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          mx0 = max3(mx0, __uint_as_float(a[i]), __uint_as_float(a[i + 1]));
+          mx1 = max3(mx1, __uint_as_float(a[i + 2]), __uint_as_float(a[i + 3]));
+          mx2 = max3(mx2, __uint_as_float(bb[i]), __uint_as_float(bb[i + 1]));
+          mx3 = max3(mx3, __uint_as_float(bb[i + 2]), __uint_as_float(bb[i + 3]));
+        }
       }
       const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
       const float m_new = fmaxf(m_used, m_tile);
@@ -327,7 +334,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orow[32];
             tmem_ld32(tO + c * 32, orow);
-            tmem_wait_ld();
+            tmem_wait_ld_regs(orow);
 #pragma unroll
             for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
             tmem_st32(tO + c * 32, orow);
@@ -336,20 +343,49 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      float l0 = 0.f, l1 = 0.f;
-      uint32_t pk[64];
+      // pass 2: p = 2^(s * scale * log2 e - m) per 32-column chunk; the chunk's 16 packed bf16
+      // columns of P go to TMEM columns [16c, 16c+16), which earlier chunks have already read.
+      // Pairs use packed fp32; every fourth pair goes to the FMA pipe (polynomial) and the rest
+      // to the MUFU, so neither unit alone paces the tile.
+      const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      uint32_t cur[32];
+      tmem_ld32(tS, cur);
+      tmem_wait_ld_regs(cur);
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[i]), p.scale_log2, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[i + 1]), p.scale_log2, neg_m));
-        l0 += p0;
-        l1 += p1;
-        pk[i >> 1] = pack_bf16x2(p0, p1);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t nxt[32];
+        if (c < 3) tmem_ld32(tS + (c + 1) * 32, nxt);  // in flight while chunk c is computed
+        if (lim < 128) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= lim) cur[i] = __float_as_uint(-INFINITY);
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 x = fma2(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), c2, nm2);
+          float2 e;
+          if ((i & 3) == 3) {
+            e = exp2_poly2(x);
+          } else {
+            e.x = ex2_approx(x.x);
+            e.y = ex2_approx(x.y);
+          }
+          if (i & 1) acc1 = add2(acc1, e);
+          else acc0 = add2(acc0, e);
+          pk[i] = pack_bf16x2(e.x, e.y);
+        }
+        tmem_st16(tS + c * 16, pk);
+        if (c < 3) {
+          tmem_wait_ld_regs(nxt);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
+        }
       }
-      l += l0 + l1;
+      l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
       if (r == 0) ATTN_TRACE_AT(2 + slot, 3, j);
-      tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       if (r == 0) ATTN_TRACE_AT(2 + slot, 4, j);
       tc_fence_before();

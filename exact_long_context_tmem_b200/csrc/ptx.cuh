@@ -190,6 +190,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// wait::ld that also names the loaded registers, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 32 consecutive columns of 32-bit: thread i of the warp gets lane (base lane + i).
@@ -268,6 +280,71 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
 // base is 1024-byte aligned (rows are 128 bytes).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// ---------------------------------------------------------------- register split
+
+// Warpgroup-wide change of the per-thread register budget.  The increases of some warpgroups
+// must be covered by the decreases of others within the block's launch allocation.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------- packed fp32 (two lanes per op)
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t mov.b64 b, {%4, %5};\n\t mov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\t mov.b64 {%0, %1}, d;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t mov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\t mov.b64 {%0, %1}, d;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two values on the FMA pipe instead of the MUFU: x = j + f with j = rint(x) and
+// f in [-0.5, 0.5]; 2^f by a degree-5 polynomial fitted here for minimum relative error on that
+// interval (max relative error 1.7e-7 when evaluated in float32, the accuracy class of
+// ex2.approx); 2^j is added to the
+// exponent field as an integer.  x is clamped at -127, where the construction yields exactly
+// +0.0, so masked scores (-inf) give 0 as the hardware ex2 does.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer in the low bits
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  const float2 t = add2(x, make_float2(kRound, kRound));
+  const float2 j = add2(t, make_float2(-kRound, -kRound));
+  const float2 f = add2(x, make_float2(-j.x, -j.y));
+  float2 q = fma2(make_float2(1.3264722656458616e-3f, 1.3264722656458616e-3f), f,
+                  make_float2(9.671512991189957e-3f, 9.671512991189957e-3f));
+  q = fma2(q, f, make_float2(5.550733581185341e-2f, 5.550733581185341e-2f));
+  q = fma2(q, f, make_float2(2.4022242426872253e-1f, 2.4022242426872253e-1f));
+  q = fma2(q, f, make_float2(6.931470036506653e-1f, 6.931470036506653e-1f));
+  q = fma2(q, f, make_float2(1.0f, 1.0f));
+  const uint32_t rx = __float_as_uint(q.x) + (__float_as_uint(t.x) << 23);
+  const uint32_t ry = __float_as_uint(q.y) + (__float_as_uint(t.y) << 23);
+  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 // ---------------------------------------------------------------- math helpers

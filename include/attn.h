@@ -223,6 +223,9 @@ ATTN_API attn_status_t attn_set_wait_limit_ns(unsigned long long ns);
  * limit; the wait runs out, the kernel records ATTN_ERR_TIMEOUT and returns.  Used to test
  * the timeout path without faulting or hanging the GPU.  Synchronises the device. */
 ATTN_API attn_status_t attn_debug_wait_probe(unsigned long long limit_ns);
+/* Evaluates the kernels' exp2 on n device floats: mode 0 = the FMA-pipe polynomial the prefill
+ * softmax uses for a quarter of its exponentials, mode 1 = the MUFU ex2.approx.  For tests. */
+ATTN_API attn_status_t attn_debug_exp2(const float* x, float* y, long long n, int mode, void* stream);
 /* Host-side fault injection for the streamer: the nth (1-based) host->device copy (what = 1)
  * or device allocation (what = 2) of the next attn_chunked_stream call fails with
  * ATTN_ERR_INJECTED.  what = 0 disarms. */
