@@ -169,16 +169,28 @@ static size_t decode_ws_bytes(const attn_dims_t& d, int P) {
   return rows * d.D * sizeof(float) + rows * sizeof(float) + 256;
 }
 
+template <bool FP8, int GP>
+static attn_status_t launch_decode_gp(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p,
+                                      dim3 grid, cudaStream_t stream) {
+  static std::atomic<uint64_t> smem_done{0};
+  if (FP8) {
+    attn_status_t st = ensure_smem(decode_fp8_sm100<GP>, DecodeFp8Cfg::SMEM_BYTES, smem_done);
+    if (st != ATTN_OK) return st;
+    decode_fp8_sm100<GP><<<grid, DecodeFp8Cfg::THREADS, DecodeFp8Cfg::SMEM_BYTES, stream>>>(mk, mv, p);
+  } else {
+    attn_status_t st = ensure_smem(decode_split_sm100<GP>, DecodeCfg::SMEM_BYTES, smem_done);
+    if (st != ATTN_OK) return st;
+    decode_split_sm100<GP><<<grid, DecodeCfg::THREADS, DecodeCfg::SMEM_BYTES, stream>>>(mk, mv, p);
+  }
+  ATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
 template <bool FP8>
 static attn_status_t launch_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
                                    const int* kv_lens, int Tmax, const attn_dims_t& d, int P, int split_tokens,
                                    void* o, float* lse, void* ws, cudaStream_t stream) {
-  static std::atomic<uint64_t> smem_done{0};
-  const int smem_bytes = FP8 ? DecodeFp8Cfg::SMEM_BYTES : DecodeCfg<false>::SMEM_BYTES;
-  const int threads = FP8 ? DecodeFp8Cfg::THREADS : DecodeCfg<false>::THREADS;
-  attn_status_t st = FP8 ? ensure_smem(decode_fp8_sm100, smem_bytes, smem_done)
-                         : ensure_smem(decode_split_sm100<false>, smem_bytes, smem_done);
-  if (st != ATTN_OK) return st;
+  attn_status_t st;
   CUtensorMap mk, mv;
   // With Tmax == 0 every split is empty and no map is read; it still needs a valid base and extent.
   const uint64_t dk[4] = {128, (uint64_t)d.Hkv, (uint64_t)std::max(Tmax, 1), (uint64_t)d.B};
@@ -213,9 +225,13 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   dim3 grid(P, d.Hkv, d.B);
-  if (FP8) decode_fp8_sm100<<<grid, threads, smem_bytes, stream>>>(mk, mv, p);
-  else decode_split_sm100<false><<<grid, threads, smem_bytes, stream>>>(mk, mv, p);
-  ATTN_CUDA(cudaGetLastError());
+  // The query group is padded to the next power of two (<= 16) so the kernels' per-row loops unroll.
+  if (p.G <= 1) st = launch_decode_gp<FP8, 1>(mk, mv, p, grid, stream);
+  else if (p.G <= 2) st = launch_decode_gp<FP8, 2>(mk, mv, p, grid, stream);
+  else if (p.G <= 4) st = launch_decode_gp<FP8, 4>(mk, mv, p, grid, stream);
+  else if (p.G <= 8) st = launch_decode_gp<FP8, 8>(mk, mv, p, grid, stream);
+  else st = launch_decode_gp<FP8, 16>(mk, mv, p, grid, stream);
+  if (st != ATTN_OK) return st;
   if (P > 1) {
     MergeParams mp{};
     mp.o_parts = p.o_part;
@@ -427,6 +443,15 @@ attn_status_t attn_set_wait_limit_ns(unsigned long long ns) {
   ATTN_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
   return ATTN_OK;
 }
+
+#ifdef ATTN_PROF
+// Profile builds only: point the cycle counters at a device buffer of 64 unsigned 64-bit words.
+ATTN_API attn_status_t attn_debug_set_prof(void* dev_ptr) {
+  unsigned long long* p = static_cast<unsigned long long*>(dev_ptr);
+  ATTN_CUDA(cudaMemcpyToSymbol(g_prof, &p, sizeof(p)));
+  return ATTN_OK;
+}
+#endif
 
 #ifdef ATTN_TRACE
 // Trace builds only: point the progress trace at host-mapped memory (device address).

@@ -18,7 +18,8 @@
 // float32-level accuracy; the dequant scales never touch the MMA operands.
 //
 // Roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer,
-// warps 2..5 softmax / conversion / epilogue (128 threads).
+// warps 2..5 softmax / epilogue (128 threads).  The query group is padded to GP (a power of two
+// <= 16, a template parameter) so the per-row loops unroll and run side by side.
 #pragma once
 
 #include "ptx.cuh"
@@ -40,30 +41,196 @@ struct DecodeParams {
   float* lse;               // [B, Hq] or null
 };
 
-template <bool FP8>
 struct DecodeCfg {
   static constexpr int D = 128;
-  static constexpr int NST = FP8 ? 4 : 3;
-  static constexpr int KV_TILE = FP8 ? 128 * 128 : 2 * 128 * 128;  // bytes of one K (or V) tile as loaded
-  static constexpr int CONV_TILE = 2 * 128 * 128;                  // f16 tile converted from codes
-  static constexpr int QBOX = 16 * 128;                            // 16 rows x 64 16-bit elements
+  static constexpr int NST = 3;
+  static constexpr int KV_TILE = 2 * 128 * 128;  // bytes of one bf16 K (or V) tile: two 64-wide boxes
+  static constexpr int QBOX = 16 * 128;          // 16 rows x 64 16-bit elements
   static constexpr int Q_BYTES = 2 * QBOX;
-  static constexpr int NQ = FP8 ? 2 : 1;
-  static constexpr int P_BYTES = 2 * QBOX;  // P^T: 16 rows x 128 tokens
+  static constexpr int P_BYTES = 2 * QBOX;       // P^T: 16 rows x 128 tokens
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NST * KV_TILE;
-  static constexpr int OFF_KC = OFF_V + NST * KV_TILE;
-  static constexpr int OFF_VC = OFF_KC + (FP8 ? CONV_TILE : 0);
-  static constexpr int OFF_Q = OFF_VC + (FP8 ? CONV_TILE : 0);
-  static constexpr int OFF_P = OFF_Q + NQ * Q_BYTES;
+  static constexpr int OFF_Q = OFF_V + NST * KV_TILE;
+  static constexpr int OFF_P = OFF_Q + Q_BYTES;
   static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;  // [2][4 warps][16] maxima + [4][16] sums
   static constexpr int OFF_BAR = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;
-  static constexpr int N_BARS = 4 * NST + 1 + 2 + 2 + 1 + 1 + 1 + 2 + 1;
+  static constexpr int N_BARS = 4 * NST + 1 + 2 + 2 + 1 + 1 + 2 + 1 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
   static constexpr int THREADS = 192;
   static constexpr uint32_t TMEM_COLS = 64;  // S^T double buffer (2 x 16) + O^T (16)
   static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
+
+// Order-preserving integer image of a float (an involution), so a warp max is one redux.sync.
+__device__ __forceinline__ int float_to_ordered(float f) {
+  const int i = __float_as_int(f);
+  return i ^ ((i >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float ordered_to_float(int i) { return __int_as_float(i ^ ((i >> 31) & 0x7fffffff)); }
+__device__ __forceinline__ float warp_max_redux(float v) {
+  int r;
+  asm volatile("redux.sync.max.s32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(float_to_ordered(v)));
+  return ordered_to_float(r);
+}
+
+template <int GP>
+struct DecodeRows {
+  float m_used[GP];  // log2-domain reference max per query row (lazy: moves by > threshold only)
+  float l_part[GP];  // this thread's share of the row sums, relative to m_used
+};
+
+// One tile of the decode softmax on the thread that owns token t (= TMEM lane t of S^T and, for
+// the O^T rescale, output element d = t).  Scores -> row maxima (warp redux, then a bounded
+// cross-warp exchange) -> lazy O rescale -> this token's entries of P^T (scaled by vs).
+// Returns false, warp-uniformly, if a bounded wait ran out.
+template <int GP, bool F16P>
+__device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j, int lane, int wq, int t,
+                                                    bool valid, float sc, float vs, uint32_t tS_lane,
+                                                    uint32_t tO_lane, float* red_max, uint64_t* red_bar,
+                                                    uint64_t* o_ready, uint8_t* p_tile, float threshold) {
+  uint32_t sv[16];
+  tmem_ld16(tS_lane, sv);
+  tmem_wait_ld();
+  float x[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
+  float* rm = red_max + (j & 1) * 64;
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float m = warp_max_redux(x[g]);
+    if (lane == 0) rm[wq * 16 + g] = m;
+  }
+  mbar_arrive(&red_bar[j & 1]);
+  if (!mbar_wait_warp(&red_bar[j & 1], (j >> 1) & 1, SITE_DC_SM_S)) return false;
+  bool need = false;
+  float alpha[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float tm = fmaxf(fmaxf(rm[g], rm[16 + g]), fmaxf(rm[32 + g], rm[48 + g]));
+    const float mn = fmaxf(rows.m_used[g], tm);
+    alpha[g] = 1.f;
+    if (mn > rows.m_used[g] + threshold) {  // the same decision on every thread of the CTA
+      alpha[g] = ex2_approx(rows.m_used[g] - mn);
+      rows.m_used[g] = mn;
+      rows.l_part[g] *= alpha[g];
+      need = true;
+    }
+  }
+  if (need && j > 0) {  // rescale O^T row t once PV(j-1) is done
+    if (!mbar_wait_warp(o_ready, (j - 1) & 1, SITE_DC_SM_O)) return false;
+    tc_fence_after();
+    uint32_t orow[16];
+    tmem_ld16(tO_lane, orow);
+    tmem_wait_ld();
+#pragma unroll
+    for (int g = 0; g < GP; ++g) orow[g] = __float_as_uint(__uint_as_float(orow[g]) * alpha[g]);
+    tmem_st16(tO_lane, orow);
+    tmem_wait_st();
+  }
+  uint8_t* prow = p_tile + (t >> 6) * (16 * 128);
+  const uint32_t pchunk = (t & 63) >> 3, pbyte = (t & 7) * 2;
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float pr = (x[g] == -INFINITY) ? 0.f : ex2_approx(x[g] - rows.m_used[g]);
+    rows.l_part[g] += pr;
+    const float pv = pr * vs;
+    const uint16_t bits = F16P ? __half_as_ushort(__float2half_rn(pv)) : __bfloat16_as_ushort(__float2bfloat16_rn(pv));
+    *reinterpret_cast<uint16_t*>(prow + sw128_offset(g, pchunk) + pbyte) = bits;
+  }
+  return true;
+}
+
+// Epilogue shared by the decode kernels: reduce the row sums over the warpgroup, wait for the last
+// PV, then thread t (= output element d) writes o[g][t] = O^T[t][g] / l_g and, for t < G, lse_t.
+// The last PV is awaited on its own single-phase barrier: on the per-tile barrier, two phases can
+// still be pending here, and a parity wait could be satisfied by the older one.
+template <int GP>
+__device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const DecodeParams& p, int G, int split,
+                                                int kvh, int b, int lane, int wq, int t, uint32_t tO_lane,
+                                                float* red_sum, uint64_t* sum_bar, uint64_t* o_final) {
+  constexpr int D = 128;
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float s = warp_sum(rows.l_part[g]);
+    if (lane == 0) red_sum[wq * 16 + g] = s;
+  }
+  mbar_arrive(sum_bar);
+  if (!mbar_wait_warp(sum_bar, 0, SITE_DC_SM_S)) return false;
+  if (!mbar_wait_warp(o_final, 0, SITE_DC_SM_O)) return false;
+  tc_fence_after();
+  uint32_t orow[16];
+  tmem_ld16(tO_lane, orow);
+  tmem_wait_ld();
+  float my_lse = -INFINITY;
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    if (g < G) {
+      const float l = red_sum[g] + red_sum[16 + g] + red_sum[32 + g] + red_sum[48 + g];
+      const float ov = (l > 0.f) ? __uint_as_float(orow[g]) / l : 0.f;
+      const float lse = (l > 0.f) ? (rows.m_used[g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (g == t) my_lse = lse;
+      const long long h = (long long)kvh * G + g;
+      if (p.n_splits == 1) {
+        p.o[((long long)b * p.Hq + h) * D + t] = __float2bfloat16_rn(ov);
+      } else {
+        p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + t] = ov;
+      }
+    }
+  }
+  if (t < G) {
+    const long long h = (long long)kvh * G + t;
+    if (p.n_splits == 1) {
+      if (p.lse) p.lse[(long long)b * p.Hq + h] = my_lse;
+    } else {
+      p.lse_part[((long long)split * p.B + b) * p.Hq + h] = my_lse;
+    }
+  }
+  return true;
+}
+
+// Empty split: o = 0, lse = -inf (written by the whole CTA, before any barrier or TMEM use).
+__device__ __forceinline__ void decode_write_empty(const DecodeParams& p, int G, int split, int kvh, int b) {
+  constexpr int D = 128;
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int g = i / D, d = i % D;
+    const long long h = (long long)kvh * G + g;
+    if (p.n_splits == 1) {
+      p.o[((long long)b * p.Hq + h) * D + d] = __float2bfloat16_rn(0.f);
+      if (d == 0 && p.lse) p.lse[(long long)b * p.Hq + h] = -INFINITY;
+    } else {
+      p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + d] = 0.f;
+      if (d == 0) p.lse_part[((long long)split * p.B + b) * p.Hq + h] = -INFINITY;
+    }
+  }
+}
+
+// Q^T rows of the group into the 16-row, 128B-swizzled B operand (rows >= G zero).  With f16_split,
+// Q is written as f16 hi at q_smem and f16 lo at q_smem + 4096; else as bf16 at q_smem.
+__device__ __forceinline__ void decode_stage_q(const DecodeParams& p, int G, int kvh, int b, int wg_tid,
+                                               uint8_t* q_smem, bool f16_split) {
+  constexpr int D = 128, QBOX = 16 * 128;
+  for (int c = wg_tid; c < 256; c += 128) {
+    const int g = c >> 4, cc = c & 15;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (g < G) x = *reinterpret_cast<const uint4*>(p.q + ((long long)b * p.Hq + (long long)kvh * G + g) * D + cc * 8);
+    const uint32_t off = (cc >> 3) * QBOX + sw128_offset(g, cc & 7);
+    if (!f16_split) {
+      *reinterpret_cast<uint4*>(q_smem + off) = x;
+    } else {
+      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float f0 = __uint_as_float(xw[i] << 16), f1 = __uint_as_float(xw[i] & 0xFFFF0000u);
+        const __half h0 = __float2half_rn(f0), h1 = __float2half_rn(f1);
+        hi[i] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+        lo[i] = pack_f16x2(f0 - __half2float(h0), f1 - __half2float(h1));
+      }
+      *reinterpret_cast<uint4*>(q_smem + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(q_smem + 2 * QBOX + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+}
 
 // Convert one token row (128 E4M3 codes, 128B-swizzled row `t` of the code tile) to f16 in the
 // two 64-wide boxes of the converted tile; invalid tokens become zeros.
@@ -89,12 +256,11 @@ __device__ __forceinline__ void convert_row_e4m3(const uint8_t* codes_tile, uint
   }
 }
 
-template <bool FP8>
+template <int GP>
 __global__ void __launch_bounds__(192, 1)
     decode_split_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const DecodeParams p) {
-  using C = DecodeCfg<FP8>;
-  constexpr int D = C::D;
+  using C = DecodeCfg;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int len = p.kv_lens[b];
@@ -103,19 +269,8 @@ __global__ void __launch_bounds__(192, 1)
   const int t1 = min(len, t0 + p.split_tokens);
   const int n = t1 > t0 ? (t1 - t0 + 127) / 128 : 0;
   const int G = p.G;
-
-  if (n == 0) {  // empty split: o = 0, lse = -inf
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-      const int g = i / D, d = i % D;
-      const long long h = (long long)kvh * G + g;
-      if (p.n_splits == 1) {
-        p.o[((long long)b * p.Hq + h) * D + d] = __float2bfloat16_rn(0.f);
-        if (d == 0 && p.lse) p.lse[(long long)b * p.Hq + h] = -INFINITY;
-      } else {
-        p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + d] = 0.f;
-        if (d == 0) p.lse_part[((long long)split * p.B + b) * p.Hq + h] = -INFINITY;
-      }
-    }
+  if (n == 0) {
+    decode_write_empty(p, G, split, kvh, b);
     return;
   }
 
@@ -130,32 +285,31 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* s_full = q_ready + 1;  // [2]
   uint64_t* p_full = s_full + 2;   // [2]
   uint64_t* o_ready = p_full + 2;
-  uint64_t* kc_ready = o_ready + 1;
-  uint64_t* drain = kc_ready + 1;
+  uint64_t* drain = o_ready + 1;
   uint64_t* red_bar = drain + 1;  // [2] cross-warp exchange of the tile maxima
   uint64_t* sum_bar = red_bar + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sum_bar + 1);
+  uint64_t* o_final = sum_bar + 1;  // single phase: every PV of the split has completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_final + 1);
   float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][16]
   float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], FP8 ? 128 : 1);
+      mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], FP8 ? 128 : 1);
+      mbar_init(&v_empty[i], 1);
     }
     mbar_init(q_ready, 128);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
+      mbar_init(&red_bar[s], 128);
     }
     mbar_init(o_ready, 1);
-    mbar_init(kc_ready, 128);
     mbar_init(drain, 1);
-    mbar_init(&red_bar[0], 128);
-    mbar_init(&red_bar[1], 128);
     mbar_init(sum_bar, 128);
+    mbar_init(o_final, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -181,21 +335,13 @@ __global__ void __launch_bounds__(192, 1)
         const int tok = t0 + j * 128;
         if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, SITE_DC_LOAD_EMPTY))) break;
         mbar_arrive_expect_tx(&k_full[st], C::KV_TILE);
-        if (FP8) {
-          tma_load_4d(smem + C::OFF_K + st * C::KV_TILE, &tmK, &k_full[st], 0, kvh, tok, b);
-        } else {
-          tma_load_4d(smem + C::OFF_K + st * C::KV_TILE, &tmK, &k_full[st], 0, kvh, tok, b);
-          tma_load_4d(smem + C::OFF_K + st * C::KV_TILE + 128 * 128, &tmK, &k_full[st], 64, kvh, tok, b);
-        }
+        tma_load_4d(smem + C::OFF_K + st * C::KV_TILE, &tmK, &k_full[st], 0, kvh, tok, b);
+        tma_load_4d(smem + C::OFF_K + st * C::KV_TILE + 128 * 128, &tmK, &k_full[st], 64, kvh, tok, b);
         issued = 2 * j + 1;
         if (!(ok = mbar_wait(&v_empty[st], ph ^ 1, SITE_DC_LOAD_EMPTY))) break;
         mbar_arrive_expect_tx(&v_full[st], C::KV_TILE);
-        if (FP8) {
-          tma_load_4d(smem + C::OFF_V + st * C::KV_TILE, &tmV, &v_full[st], 0, kvh, tok, b);
-        } else {
-          tma_load_4d(smem + C::OFF_V + st * C::KV_TILE, &tmV, &v_full[st], 0, kvh, tok, b);
-          tma_load_4d(smem + C::OFF_V + st * C::KV_TILE + 128 * 128, &tmV, &v_full[st], 64, kvh, tok, b);
-        }
+        tma_load_4d(smem + C::OFF_V + st * C::KV_TILE, &tmV, &v_full[st], 0, kvh, tok, b);
+        tma_load_4d(smem + C::OFF_V + st * C::KV_TILE + 128 * 128, &tmV, &v_full[st], 64, kvh, tok, b);
         issued = 2 * j + 2;
       }
       if (!ok) {
@@ -210,22 +356,21 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = make_idesc_f16(128, 16, false, false, !FP8);
-      constexpr uint32_t idesc_pv = make_idesc_f16(128, 16, true, false, !FP8);
+      constexpr uint32_t idesc_qk = make_idesc_f16(128, 16, false, false, true);
+      constexpr uint32_t idesc_pv = make_idesc_f16(128, 16, true, false, true);
       const uint32_t sQ = smem_u32(smem + C::OFF_Q);
       const uint32_t sP = smem_u32(smem + C::OFF_P);
-      // S^T(j) = K_j . Q^T into S buffer `buf`; `kbase` is the K tile (loaded or converted).
-      auto issue_s = [&](uint32_t kbase, int buf) {
-        constexpr int KSTEPS = FP8 ? 16 : 8;  // FP8: Q hi then Q lo over the same K columns
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-          const int kd = kk & 7;
-          const uint32_t koff = (kd >> 2) * (128 * 128) + (kd & 3) * 32;
-          const uint32_t qoff = (kk >> 3) * C::Q_BYTES + (kd >> 2) * C::QBOX + (kd & 3) * 32;
+      const uint32_t sK = smem_u32(smem + C::OFF_K);
+      const uint32_t sV = smem_u32(smem + C::OFF_V);
+      auto issue_s = [&](uint32_t kbase, int buf) {  // S^T(j) = K_j . Q^T
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * C::QBOX + (kk & 3) * 32;
           mma_ss(tS0 + buf * 16, make_sdesc_sw128(kbase + koff, 16, 1024), make_sdesc_sw128(sQ + qoff, 16, 1024),
                  idesc_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](uint32_t vbase, int pbuf, bool acc) {
+      auto issue_pv = [&](uint32_t vbase, int pbuf, bool acc) {  // O^T += V_j^T . P_j^T
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t da = make_sdesc_sw128(vbase + kk * 16 * 128, 128 * 128, 1024);
           const uint64_t db =
@@ -233,48 +378,32 @@ __global__ void __launch_bounds__(192, 1)
           mma_ss(tO, da, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      const uint32_t sK = smem_u32(smem + C::OFF_K);
-      const uint32_t sV = smem_u32(smem + C::OFF_V);
       bool ok = mbar_wait(q_ready, 0, SITE_DC_MMA_K);
-      if (!FP8) {
-        for (int jj = 0; jj < 2 && jj < n && ok; ++jj) {
-          if (!(ok = mbar_wait(&k_full[jj % C::NST], (jj / C::NST) & 1, SITE_DC_MMA_K))) break;
+      for (int jj = 0; jj < 2 && jj < n && ok; ++jj) {
+        if (!(ok = mbar_wait(&k_full[jj % C::NST], (jj / C::NST) & 1, SITE_DC_MMA_K))) break;
+        tc_fence_after();
+        issue_s(sK + (jj % C::NST) * C::KV_TILE, jj & 1);
+        mma_commit(&s_full[jj & 1]);
+        mma_commit(&k_empty[jj % C::NST]);
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j % C::NST;
+        if (!(ok = mbar_wait(&v_full[st], (j / C::NST) & 1, SITE_DC_MMA_V))) break;
+        if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, SITE_DC_MMA_P))) break;
+        tc_fence_after();
+        issue_pv(sV + st * C::KV_TILE, j & 1, j > 0);
+        mma_commit(o_ready);
+        mma_commit(&v_empty[st]);
+        if (j + 2 < n) {
+          const int st2 = (j + 2) % C::NST;
+          if (!(ok = mbar_wait(&k_full[st2], ((j + 2) / C::NST) & 1, SITE_DC_MMA_K))) break;
           tc_fence_after();
-          issue_s(sK + (jj % C::NST) * C::KV_TILE, jj & 1);
-          mma_commit(&s_full[jj & 1]);
-          mma_commit(&k_empty[jj % C::NST]);
-        }
-        for (int j = 0; j < n && ok; ++j) {
-          const int st = j % C::NST;
-          if (!(ok = mbar_wait(&v_full[st], (j / C::NST) & 1, SITE_DC_MMA_V))) break;
-          if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, SITE_DC_MMA_P))) break;
-          tc_fence_after();
-          issue_pv(sV + st * C::KV_TILE, j & 1, j > 0);
-          mma_commit(o_ready);
-          mma_commit(&v_empty[st]);
-          if (j + 2 < n) {
-            const int st2 = (j + 2) % C::NST;
-            if (!(ok = mbar_wait(&k_full[st2], ((j + 2) / C::NST) & 1, SITE_DC_MMA_K))) break;
-            tc_fence_after();
-            issue_s(sK + st2 * C::KV_TILE, j & 1);
-            mma_commit(&s_full[j & 1]);
-            mma_commit(&k_empty[st2]);
-          }
-        }
-      } else {
-        const uint32_t sKc = smem_u32(smem + C::OFF_KC);
-        const uint32_t sVc = smem_u32(smem + C::OFF_VC);
-        for (int j = 0; j < n && ok; ++j) {
-          if (!(ok = mbar_wait(kc_ready, j & 1, SITE_DC_MMA_K))) break;
-          tc_fence_after();
-          issue_s(sKc, j & 1);
+          issue_s(sK + st2 * C::KV_TILE, j & 1);
           mma_commit(&s_full[j & 1]);
-          if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, SITE_DC_MMA_P))) break;
-          tc_fence_after();
-          issue_pv(sVc, j & 1, j > 0);
-          mma_commit(o_ready);
+          mma_commit(&k_empty[st2]);
         }
       }
+      if (ok) mma_commit(o_final);
       mma_commit(drain);
       mbar_wait_drain(drain, 0, SITE_DC_DRAIN);
     }
@@ -285,131 +414,34 @@ __global__ void __launch_bounds__(192, 1)
     const int t = wq * 32 + lane;  // token of the tile / TMEM lane / output element d
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int wg_tid = threadIdx.x - 64;
-    // P^T buffers: rows >= G stay zero.
-    for (int i = wg_tid; i < 2 * C::P_BYTES / 16; i += 128)
+    for (int i = wg_tid; i < 2 * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
-    // Q^T: 16 rows (G real) x 128, two 64-wide boxes, 128B swizzle.
-    for (int c = wg_tid; c < 256; c += 128) {
-      const int g = c >> 4, cc = c & 15;
-      uint4 x = make_uint4(0u, 0u, 0u, 0u);
-      if (g < G) x = *reinterpret_cast<const uint4*>(p.q + ((long long)b * p.Hq + (long long)kvh * G + g) * D + cc * 8);
-      const uint32_t off = (cc >> 3) * C::QBOX + sw128_offset(g, cc & 7);
-      if (!FP8) {
-        *reinterpret_cast<uint4*>(smem + C::OFF_Q + off) = x;
-      } else {
-        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float f0 = __uint_as_float(xw[i] << 16), f1 = __uint_as_float(xw[i] & 0xFFFF0000u);
-          const __half h0 = __float2half_rn(f0), h1 = __float2half_rn(f1);
-          hi[i] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-          lo[i] = pack_f16x2(f0 - __half2float(h0), f1 - __half2float(h1));
-        }
-        *reinterpret_cast<uint4*>(smem + C::OFF_Q + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(smem + C::OFF_Q + C::Q_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-    }
+    decode_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, false);
     fence_proxy_async_smem();
     mbar_arrive(q_ready);
 
-    float m_used[16], l_part[16];
+    DecodeRows<GP> rows;
 #pragma unroll
-    for (int g = 0; g < 16; ++g) {
-      m_used[g] = -INFINITY;
-      l_part[g] = 0.f;
+    for (int g = 0; g < GP; ++g) {
+      rows.m_used[g] = -INFINITY;
+      rows.l_part[g] = 0.f;
     }
     bool ok = true;
-    const long long kv_row0 = (long long)b * p.Tmax;
-    if (FP8) {  // convert K_0
-      ok = mbar_wait_warp(&k_full[0], 0, SITE_DC_SM_K);
-      if (ok) {
-        convert_row_e4m3(smem + C::OFF_K, smem + C::OFF_KC, t, t0 + t < t1);
-        mbar_arrive(&k_empty[0]);
-        fence_proxy_async_smem();
-        mbar_arrive(kc_ready);
-      }
-    }
     for (int j = 0; j < n && ok; ++j) {
       const int st = j % C::NST;
       const uint32_t ph = (j / C::NST) & 1;
-      const int tok = t0 + j * 128 + t;
-      const bool valid = tok < t1;
-      float ks = 1.f, vs = 1.f;
-      if (FP8 && valid) {
-        ks = p.k_scale[(kv_row0 + tok) * p.Hkv + kvh];
-        vs = p.v_scale[(kv_row0 + tok) * p.Hkv + kvh];
-      }
+      const bool valid = t0 + j * 128 + t < t1;
       // tcgen05.ld/st are warp-collective: every lane takes the same branch around them.
       if (!(ok = mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
       tc_fence_after();
-      uint32_t sv[16];
-      tmem_ld16(tS0 + (j & 1) * 16 + lane_off, sv);
-      tmem_wait_ld();
-      float x[16];
-      const float sc = p.scale_log2 * ks;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
-      float* rm = red_max + (j & 1) * 64;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float m = warp_max(x[g]);
-          if (lane == 0) rm[wq * 16 + g] = m;
-        }
-      }
-      mbar_arrive(&red_bar[j & 1]);
-      if (!(ok = mbar_wait_warp(&red_bar[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
-      bool need = false;
-      float alpha[16];
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        alpha[g] = 1.f;
-        if (g < G) {
-          const float tm = fmaxf(fmaxf(rm[g], rm[16 + g]), fmaxf(rm[32 + g], rm[48 + g]));
-          const float mn = fmaxf(m_used[g], tm);
-          if (mn > m_used[g] + C::RESCALE_THRESHOLD) {
-            alpha[g] = ex2_approx(m_used[g] - mn);
-            m_used[g] = mn;
-            l_part[g] *= alpha[g];
-            need = true;
-          }
-        }
-      }
-      if (need && j > 0) {  // rescale O^T row t (element d = t of every query row)
-        if (!(ok = mbar_wait_warp(o_ready, (j - 1) & 1, SITE_DC_SM_O))) break;
-        tc_fence_after();
-        uint32_t orow[16];
-        tmem_ld16(tO + lane_off, orow);
-        tmem_wait_ld();
-#pragma unroll
-        for (int g = 0; g < 16; ++g) orow[g] = __float_as_uint(__uint_as_float(orow[g]) * alpha[g]);
-        tmem_st16(tO + lane_off, orow);
-        tmem_wait_st();
-      }
-      uint8_t* prow = smem + C::OFF_P + (j & 1) * C::P_BYTES + (t >> 6) * C::QBOX;
-      const uint32_t pchunk = (t & 63) >> 3, pbyte = (t & 7) * 2;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float pr = (x[g] == -INFINITY) ? 0.f : ex2_approx(x[g] - m_used[g]);
-          l_part[g] += pr;
-          const float pv = pr * vs;
-          uint16_t bits;
-          if (FP8) bits = __half_as_ushort(__float2half_rn(pv));
-          else bits = __bfloat16_as_ushort(__float2bfloat16_rn(pv));
-          *reinterpret_cast<uint16_t*>(prow + sw128_offset(g, pchunk) + pbyte) = bits;
-        }
-      }
-      if (FP8) {
-        // V_j codes -> f16 (needs PV(j-1) finished reading the converted V tile)
-        if (j > 0 && !(ok = mbar_wait_warp(o_ready, (j - 1) & 1, SITE_DC_SM_O))) break;
-        if (!(ok = mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V))) break;
-        convert_row_e4m3(smem + C::OFF_V + st * C::KV_TILE, smem + C::OFF_VC, t, valid);
-        mbar_arrive(&v_empty[st]);
-      } else if (t1 - (t0 + j * 128) < 128) {
+      if (!(ok = decode_softmax_tile<GP, false>(rows, j, lane, wq, t, valid, p.scale_log2, 1.f,
+                                                tS0 + (j & 1) * 16 + lane_off, tO + lane_off, red_max, red_bar,
+                                                o_ready, smem + C::OFF_P + (j & 1) * C::P_BYTES,
+                                                C::RESCALE_THRESHOLD)))
+        break;
+      if (t1 - (t0 + j * 128) < 128) {
         // last, partial tile: cache slots past the length may hold anything (NaN included);
-        // zero those V rows so 0-probability x slot cannot poison the sum.
+        // zero those V rows so a 0-probability x slot product cannot poison the sum.
         if (!(ok = mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V))) break;
         if (!valid) {
           uint4* r0 = reinterpret_cast<uint4*>(smem + C::OFF_V + st * C::KV_TILE + t * 128);
@@ -421,57 +453,8 @@ __global__ void __launch_bounds__(192, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[j & 1]);
-      if (FP8 && j + 1 < n) {  // K_{j+1} codes -> f16 (S(j) has finished reading the converted K tile)
-        const int st1 = (j + 1) % C::NST;
-        if (!(ok = mbar_wait_warp(&k_full[st1], ((j + 1) / C::NST) & 1, SITE_DC_SM_K))) break;
-        convert_row_e4m3(smem + C::OFF_K + st1 * C::KV_TILE, smem + C::OFF_KC, t, tok + 128 < t1);
-        mbar_arrive(&k_empty[st1]);
-        fence_proxy_async_smem();
-        mbar_arrive(kc_ready);
-      }
     }
-    // ---- epilogue: reduce the row sums, normalise O^T, write o / lse (or the split's partial)
-    if (ok) {
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float s = warp_sum(l_part[g]);
-          if (lane == 0) red_sum[wq * 16 + g] = s;
-        }
-      }
-      mbar_arrive(sum_bar);
-      ok = mbar_wait_warp(sum_bar, 0, SITE_DC_SM_S) && mbar_wait_warp(o_ready, (n - 1) & 1, SITE_DC_SM_O);
-    }
-    if (ok) {
-      tc_fence_after();
-      uint32_t orow[16];
-      tmem_ld16(tO + lane_off, orow);
-      tmem_wait_ld();
-      float my_lse = -INFINITY;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float l = red_sum[g] + red_sum[16 + g] + red_sum[32 + g] + red_sum[48 + g];
-          const float ov = (l > 0.f) ? __uint_as_float(orow[g]) / l : 0.f;
-          const float lse = (l > 0.f) ? (m_used[g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-          if (g == t) my_lse = lse;
-          const long long h = (long long)kvh * G + g;
-          if (p.n_splits == 1) {
-            p.o[((long long)b * p.Hq + h) * D + t] = __float2bfloat16_rn(ov);
-          } else {
-            p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + t] = ov;
-          }
-        }
-      }
-      if (t < G) {
-        const long long h = (long long)kvh * G + t;
-        if (p.n_splits == 1) {
-          if (p.lse) p.lse[(long long)b * p.Hq + h] = my_lse;
-        } else {
-          p.lse_part[((long long)split * p.B + b) * p.Hq + h] = my_lse;
-        }
-      }
-    }
+    if (ok) decode_epilogue<GP>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, o_final);
   }
   tc_fence_before();
   __syncthreads();

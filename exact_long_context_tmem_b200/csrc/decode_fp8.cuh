@@ -39,13 +39,14 @@ struct DecodeFp8Cfg {
   static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;
   static constexpr int OFF_BAR = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;
-  static constexpr int N_BARS = 4 * NCS + 1 + 2 + 2 + 1 + 8 + 1 + 2 + 1;
+  static constexpr int N_BARS = 4 * NCS + 1 + 2 + 2 + 1 + 8 + 1 + 2 + 1 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
   static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
 
+template <int GP>
 __global__ void __launch_bounds__(320, 1)
     decode_fp8_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
@@ -60,18 +61,8 @@ __global__ void __launch_bounds__(320, 1)
   const int n = t1 > t0 ? (t1 - t0 + 127) / 128 : 0;
   const int G = p.G;
 
-  if (n == 0) {  // empty split: o = 0, lse = -inf
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-      const int g = i / D, d = i % D;
-      const long long h = (long long)kvh * G + g;
-      if (p.n_splits == 1) {
-        p.o[((long long)b * p.Hq + h) * D + d] = __float2bfloat16_rn(0.f);
-        if (d == 0 && p.lse) p.lse[(long long)b * p.Hq + h] = -INFINITY;
-      } else {
-        p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + d] = 0.f;
-        if (d == 0) p.lse_part[((long long)split * p.B + b) * p.Hq + h] = -INFINITY;
-      }
-    }
+  if (n == 0) {
+    decode_write_empty(p, G, split, kvh, b);
     return;
   }
 
@@ -93,7 +84,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* drain = vc_empty + 2;
   uint64_t* red_bar = drain + 1;           // [2]
   uint64_t* sum_bar = red_bar + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sum_bar + 1);
+  uint64_t* o_final = sum_bar + 1;  // single phase: every PV of the split has completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_final + 1);
   float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][16]
   float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
 
@@ -117,6 +109,7 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(o_ready, 1);
     mbar_init(drain, 1);
     mbar_init(sum_bar, 128);
+    mbar_init(o_final, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -181,6 +174,9 @@ __global__ void __launch_bounds__(320, 1)
           mma_ss(tO, da, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
+      ATTN_PROF_DECL(pw_vc);
+      ATTN_PROF_DECL(pw_p);
+      ATTN_PROF_DECL(pw_kc);
       bool ok = mbar_wait(q_ready, 0, SITE_DC_MMA_K);
       for (int jj = 0; jj < 2 && jj < n && ok; ++jj) {
         if (!(ok = mbar_wait(&kc_full[jj], 0, SITE_DC_MMA_K))) break;
@@ -192,22 +188,32 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; j < n && ok; ++j) {
         const int b2 = j & 1;
         const uint32_t ph2 = (j >> 1) & 1;
+        ATTN_PROF_T0(q0);
         if (!(ok = mbar_wait(&vc_full[b2], ph2, SITE_DC_MMA_V))) break;
+        ATTN_PROF_ADD(pw_vc, q0);
+        ATTN_PROF_T0(q1);
         if (!(ok = mbar_wait(&p_full[b2], ph2, SITE_DC_MMA_P))) break;
+        ATTN_PROF_ADD(pw_p, q1);
         tc_fence_after();
         issue_pv(b2, j > 0);
         mma_commit(o_ready);
         mma_commit(&vc_empty[b2]);
         if (j + 2 < n) {
+          ATTN_PROF_T0(q2);
           if (!(ok = mbar_wait(&kc_full[b2], ((j + 2) >> 1) & 1, SITE_DC_MMA_K))) break;
+          ATTN_PROF_ADD(pw_kc, q2);
           tc_fence_after();
           issue_s(b2);
           mma_commit(&s_full[b2]);
           mma_commit(&kc_empty[b2]);
         }
       }
+      if (ok) mma_commit(o_final);
       mma_commit(drain);
       mbar_wait_drain(drain, 0, SITE_DC_DRAIN);
+      ATTN_PROF_FLUSH(0, pw_vc);
+      ATTN_PROF_FLUSH(1, pw_p);
+      ATTN_PROF_FLUSH(2, pw_kc);
     }
     __syncwarp();
   } else if (warp < 6) {
@@ -215,6 +221,12 @@ __global__ void __launch_bounds__(320, 1)
     const int wq = warp & 3;
     const int t = wq * 32 + lane;  // token row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    ATTN_PROF_DECL(cw_k);
+    ATTN_PROF_DECL(cw_kce);
+    ATTN_PROF_DECL(cc_k);
+    ATTN_PROF_DECL(cw_v);
+    ATTN_PROF_DECL(cw_vce);
+    ATTN_PROF_DECL(cc_v);
     for (int j = 0; j < n; ++j) {
       const int st = j % C::NCS;
       const uint32_t ph = (j / C::NCS) & 1;
@@ -222,8 +234,13 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t ph2 = (j >> 1) & 1;
       const bool valid = t0 + j * 128 + t < t1;
       // K_j -> f16 -> TMEM lane t (64 columns, two f16 per column)
+      ATTN_PROF_T0(c0);
       if (!mbar_wait_warp(&k_full[st], ph, SITE_DC_SM_K)) break;
+      ATTN_PROF_ADD(cw_k, c0);
+      ATTN_PROF_T0(c1);
       if (!mbar_wait_warp(&kc_empty[b2], ph2 ^ 1, SITE_DC_SM_K)) break;
+      ATTN_PROF_ADD(cw_kce, c1);
+      ATTN_PROF_T0(c2);
       tc_fence_after();
       const uint8_t* ktile = smem + C::OFF_KCODE + st * C::CODE_TILE;
 #pragma unroll
@@ -247,13 +264,28 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&k_empty[st]);
       tc_fence_before();
       mbar_arrive(&kc_full[b2]);
+      ATTN_PROF_ADD(cc_k, c2);
       // V_j -> f16 in shared memory (zeros for tokens past the length)
+      ATTN_PROF_T0(c3);
       if (!mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V)) break;
+      ATTN_PROF_ADD(cw_v, c3);
+      ATTN_PROF_T0(c4);
       if (!mbar_wait_warp(&vc_empty[b2], ph2 ^ 1, SITE_DC_SM_V)) break;
+      ATTN_PROF_ADD(cw_vce, c4);
+      ATTN_PROF_T0(c5);
       convert_row_e4m3(smem + C::OFF_VCODE + st * C::CODE_TILE, smem + C::OFF_VC + b2 * C::VC_TILE, t, valid);
       mbar_arrive(&v_empty[st]);
       fence_proxy_async_smem();
       mbar_arrive(&vc_full[b2]);
+      ATTN_PROF_ADD(cc_v, c5);
+    }
+    if (lane == 0 && wq == 2) {
+      ATTN_PROF_FLUSH(3, cw_k);
+      ATTN_PROF_FLUSH(4, cw_kce);
+      ATTN_PROF_FLUSH(5, cc_k);
+      ATTN_PROF_FLUSH(6, cw_v);
+      ATTN_PROF_FLUSH(7, cw_vce);
+      ATTN_PROF_FLUSH(8, cc_v);
     }
   } else {
     // ------------------------------------------------------------------ softmax warpgroup
@@ -261,148 +293,59 @@ __global__ void __launch_bounds__(320, 1)
     const int t = wq * 32 + lane;  // token of the tile / TMEM lane / output element d
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int wg_tid = threadIdx.x - 192;
-    for (int i = wg_tid; i < 2 * C::P_BYTES / 16; i += 128)
+    for (int i = wg_tid; i < 2 * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
-    for (int c = wg_tid; c < 256; c += 128) {  // Q^T as f16 hi and lo, 16 rows (G real)
-      const int g = c >> 4, cc = c & 15;
-      uint4 x = make_uint4(0u, 0u, 0u, 0u);
-      if (g < G) x = *reinterpret_cast<const uint4*>(p.q + ((long long)b * p.Hq + (long long)kvh * G + g) * D + cc * 8);
-      const uint32_t off = (cc >> 3) * C::QBOX + sw128_offset(g, cc & 7);
-      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float f0 = __uint_as_float(xw[i] << 16), f1 = __uint_as_float(xw[i] & 0xFFFF0000u);
-        const __half h0 = __float2half_rn(f0), h1 = __float2half_rn(f1);
-        hi[i] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-        lo[i] = pack_f16x2(f0 - __half2float(h0), f1 - __half2float(h1));
-      }
-      *reinterpret_cast<uint4*>(smem + C::OFF_Q + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(smem + C::OFF_Q + C::Q_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
+    decode_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, true);
     fence_proxy_async_smem();
     mbar_arrive(q_ready);
 
-    float m_used[16], l_part[16];
+    DecodeRows<GP> rows;
 #pragma unroll
-    for (int g = 0; g < 16; ++g) {
-      m_used[g] = -INFINITY;
-      l_part[g] = 0.f;
+    for (int g = 0; g < GP; ++g) {
+      rows.m_used[g] = -INFINITY;
+      rows.l_part[g] = 0.f;
     }
     bool ok = true;
     const long long kv_row0 = (long long)b * p.Tmax;
+    // Per-token scales are prefetched one tile ahead so their global-memory latency stays off
+    // the tile's critical path.
+    float ks_next = 1.f, vs_next = 1.f;
+    if (t0 + t < t1) {
+      ks_next = __ldg(p.k_scale + (kv_row0 + t0 + t) * p.Hkv + kvh);
+      vs_next = __ldg(p.v_scale + (kv_row0 + t0 + t) * p.Hkv + kvh);
+    }
+    ATTN_PROF_DECL(sw_s);
+    ATTN_PROF_DECL(sc_all);
     for (int j = 0; j < n && ok; ++j) {
+      ATTN_PROF_T0(s0);
       const int b2 = j & 1;
       const uint32_t ph2 = (j >> 1) & 1;
       const int tok = t0 + j * 128 + t;
       const bool valid = tok < t1;
-      float ks = 1.f, vs = 1.f;
-      if (valid) {
-        ks = p.k_scale[(kv_row0 + tok) * p.Hkv + kvh];
-        vs = p.v_scale[(kv_row0 + tok) * p.Hkv + kvh];
+      const float ks = ks_next, vs = vs_next;
+      if (tok + 128 < t1) {
+        ks_next = __ldg(p.k_scale + (kv_row0 + tok + 128) * p.Hkv + kvh);
+        vs_next = __ldg(p.v_scale + (kv_row0 + tok + 128) * p.Hkv + kvh);
       }
+      ATTN_PROF_T0(s1);
       if (!(ok = mbar_wait_warp(&s_full[b2], ph2, SITE_DC_SM_S))) break;
+      ATTN_PROF_ADD(sw_s, s1);
       tc_fence_after();
-      uint32_t sv[16];
-      tmem_ld16(tS0 + b2 * 16 + lane_off, sv);
-      tmem_wait_ld();
-      float x[16];
-      const float sc = p.scale_log2 * ks;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
-      float* rm = red_max + b2 * 64;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float m = warp_max(x[g]);
-          if (lane == 0) rm[wq * 16 + g] = m;
-        }
-      }
-      mbar_arrive(&red_bar[b2]);
-      if (!(ok = mbar_wait_warp(&red_bar[b2], ph2, SITE_DC_SM_S))) break;
-      bool need = false;
-      float alpha[16];
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        alpha[g] = 1.f;
-        if (g < G) {
-          const float tm = fmaxf(fmaxf(rm[g], rm[16 + g]), fmaxf(rm[32 + g], rm[48 + g]));
-          const float mn = fmaxf(m_used[g], tm);
-          if (mn > m_used[g] + C::RESCALE_THRESHOLD) {
-            alpha[g] = ex2_approx(m_used[g] - mn);
-            m_used[g] = mn;
-            l_part[g] *= alpha[g];
-            need = true;
-          }
-        }
-      }
-      if (need && j > 0) {  // the decision is CTA-uniform (it follows the reduced maxima)
-        if (!(ok = mbar_wait_warp(o_ready, (j - 1) & 1, SITE_DC_SM_O))) break;
-        tc_fence_after();
-        uint32_t orow[16];
-        tmem_ld16(tO + lane_off, orow);
-        tmem_wait_ld();
-#pragma unroll
-        for (int g = 0; g < 16; ++g) orow[g] = __float_as_uint(__uint_as_float(orow[g]) * alpha[g]);
-        tmem_st16(tO + lane_off, orow);
-        tmem_wait_st();
-      }
-      uint8_t* prow = smem + C::OFF_P + b2 * C::P_BYTES + (t >> 6) * C::QBOX;
-      const uint32_t pchunk = (t & 63) >> 3, pbyte = (t & 7) * 2;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float pr = (x[g] == -INFINITY) ? 0.f : ex2_approx(x[g] - m_used[g]);
-          l_part[g] += pr;
-          *reinterpret_cast<uint16_t*>(prow + sw128_offset(g, pchunk) + pbyte) =
-              __half_as_ushort(__float2half_rn(pr * vs));
-        }
-      }
+      if (!(ok = decode_softmax_tile<GP, true>(rows, j, lane, wq, t, valid, p.scale_log2 * ks, vs,
+                                               tS0 + b2 * 16 + lane_off, tO + lane_off, red_max, red_bar, o_ready,
+                                               smem + C::OFF_P + b2 * C::P_BYTES, C::RESCALE_THRESHOLD)))
+        break;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[b2]);
+      ATTN_PROF_ADD(sc_all, s0);
     }
-    if (ok) {
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float s = warp_sum(l_part[g]);
-          if (lane == 0) red_sum[wq * 16 + g] = s;
-        }
-      }
-      mbar_arrive(sum_bar);
-      ok = mbar_wait_warp(sum_bar, 0, SITE_DC_SM_S) && mbar_wait_warp(o_ready, (n - 1) & 1, SITE_DC_SM_O);
+    if (lane == 0 && wq == 2) {
+      ATTN_PROF_FLUSH(9, sw_s);
+      ATTN_PROF_FLUSH(11, sc_all);
+      ATTN_PROF_FLUSH(12, (long long)n);
     }
-    if (ok) {
-      tc_fence_after();
-      uint32_t orow[16];
-      tmem_ld16(tO + lane_off, orow);
-      tmem_wait_ld();
-      float my_lse = -INFINITY;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        if (g < G) {
-          const float l = red_sum[g] + red_sum[16 + g] + red_sum[32 + g] + red_sum[48 + g];
-          const float ov = (l > 0.f) ? __uint_as_float(orow[g]) / l : 0.f;
-          const float lse = (l > 0.f) ? (m_used[g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-          if (g == t) my_lse = lse;
-          const long long h = (long long)kvh * G + g;
-          if (p.n_splits == 1) {
-            p.o[((long long)b * p.Hq + h) * D + t] = __float2bfloat16_rn(ov);
-          } else {
-            p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + t] = ov;
-          }
-        }
-      }
-      if (t < G) {
-        const long long h = (long long)kvh * G + t;
-        if (p.n_splits == 1) {
-          if (p.lse) p.lse[(long long)b * p.Hq + h] = my_lse;
-        } else {
-          p.lse_part[((long long)split * p.B + b) * p.Hq + h] = my_lse;
-        }
-      }
-    }
+    if (ok) decode_epilogue<GP>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, o_final);
   }
   tc_fence_before();
   __syncthreads();

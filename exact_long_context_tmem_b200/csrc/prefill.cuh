@@ -18,7 +18,15 @@
 
 #include "ptx.cuh"
 
+// One in this many exponential pairs of the softmax is computed by polynomial on the FMA pipe
+// instead of the MUFU (0: all on the MUFU).
+#ifndef ATTN_PREFILL_POLY_PERIOD
+#define ATTN_PREFILL_POLY_PERIOD 8
+#endif
+
 namespace attn {
+
+constexpr int kPolyPeriod = ATTN_PREFILL_POLY_PERIOD;
 
 struct PrefillParams {
   int B, Hq, Hkv, D, S, T, G;
@@ -296,29 +304,24 @@ __global__ void __launch_bounds__(384, 1)
         lim64 = c2 < lim64 ? c2 : lim64;
       }
       const int lim = lim64 < 0 ? 0 : (lim64 > 128 ? 128 : (int)lim64);
-      // pass 1: row max over the 128 scores, read from TMEM in two halves
+      // all 128 scores of the row in registers (one TMEM round trip)
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_wait_ld_regs(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      if (lim < 128) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= lim) sr[i] = __float_as_uint(-INFINITY);
+      }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t a[32], bb[32];
-        tmem_ld32(tS + h * 64, a);
-        tmem_ld32(tS + h * 64 + 32, bb);
-        tmem_wait_ld_regs(a);
-        tmem_wait_ld_regs(bb);
-        if (lim < 128) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (h * 64 + i >= lim) a[i] = __float_as_uint(-INFINITY);
-            if (h * 64 + 32 + i >= lim) bb[i] = __float_as_uint(-INFINITY);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          mx0 = max3(mx0, __uint_as_float(a[i]), __uint_as_float(a[i + 1]));
-          mx1 = max3(mx1, __uint_as_float(a[i + 2]), __uint_as_float(a[i + 3]));
-          mx2 = max3(mx2, __uint_as_float(bb[i]), __uint_as_float(bb[i + 1]));
-          mx3 = max3(mx3, __uint_as_float(bb[i + 2]), __uint_as_float(bb[i + 3]));
-        }
+      for (int i = 0; i < 128; i += 8) {
+        mx0 = max3(mx0, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+        mx1 = max3(mx1, __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+        mx2 = max3(mx2, __uint_as_float(sr[i + 4]), __uint_as_float(sr[i + 5]));
+        mx3 = max3(mx3, __uint_as_float(sr[i + 6]), __uint_as_float(sr[i + 7]));
       }
       const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
       const float m_new = fmaxf(m_used, m_tile);
@@ -343,31 +346,21 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      // pass 2: p = 2^(s * scale * log2 e - m) per 32-column chunk; the chunk's 16 packed bf16
-      // columns of P go to TMEM columns [16c, 16c+16), which earlier chunks have already read.
-      // Pairs use packed fp32; every fourth pair goes to the FMA pipe (polynomial) and the rest
-      // to the MUFU, so neither unit alone paces the tile.
+      // p = 2^(s * scale * log2 e - m) in packed fp32 pairs; one pair in ATTN_PREFILL_POLY_PERIOD
+      // goes to the FMA pipe (polynomial) and the rest to the MUFU.  P is stored per 32 scores (16 packed columns, over
+      // S columns already read into registers) so those registers retire early.
       const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nm2 = make_float2(neg_m, neg_m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-      uint32_t cur[32];
-      tmem_ld32(tS, cur);
-      tmem_wait_ld_regs(cur);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t nxt[32];
-        if (c < 3) tmem_ld32(tS + (c + 1) * 32, nxt);  // in flight while chunk c is computed
-        if (lim < 128) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i >= lim) cur[i] = __float_as_uint(-INFINITY);
-        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 x = fma2(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), c2, nm2);
+          const int k = c * 32 + 2 * i;
+          const float2 x = fma2(make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), c2, nm2);
           float2 e;
-          if ((i & 3) == 3) {
+          if (kPolyPeriod > 0 && i % (kPolyPeriod > 0 ? kPolyPeriod : 1) == kPolyPeriod - 1) {
             e = exp2_poly2(x);
           } else {
             e.x = ex2_approx(x.x);
@@ -378,11 +371,6 @@ __global__ void __launch_bounds__(384, 1)
           pk[i] = pack_bf16x2(e.x, e.y);
         }
         tmem_st16(tS + c * 16, pk);
-        if (c < 3) {
-          tmem_wait_ld_regs(nxt);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
-        }
       }
       l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
       if (r == 0) ATTN_TRACE_AT(2 + slot, 3, j);

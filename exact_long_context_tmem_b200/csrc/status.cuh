@@ -65,4 +65,22 @@ __device__ uint32_t* g_trace = nullptr;
   } while (0)
 #endif
 
+// Optional cycle profile (compiled in only with -DATTN_PROF): roles add clock64() spans per
+// category into a device buffer of 64 counters that the host reads after the kernel.
+#ifdef ATTN_PROF
+__device__ unsigned long long* g_prof = nullptr;
+#define ATTN_PROF_DECL(name) long long name = 0
+#define ATTN_PROF_T0(v) const long long v = clock64()
+#define ATTN_PROF_ADD(acc, t0) (acc) += clock64() - (t0)
+#define ATTN_PROF_FLUSH(slot, acc)                                    \
+  do {                                                                \
+    if (g_prof) atomicAdd(g_prof + (slot), (unsigned long long)(acc)); \
+  } while (0)
+#else
+#define ATTN_PROF_DECL(name)
+#define ATTN_PROF_T0(v)
+#define ATTN_PROF_ADD(acc, t0)
+#define ATTN_PROF_FLUSH(slot, acc)
+#endif
+
 }  // namespace attn
