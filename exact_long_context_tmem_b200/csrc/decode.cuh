@@ -82,18 +82,28 @@ struct DecodeRows {
 // One tile of the decode softmax on the thread that owns token t (= TMEM lane t of S^T and, for
 // the O^T rescale, output element d = t).  Scores -> row maxima (warp redux, then a bounded
 // cross-warp exchange) -> lazy O rescale -> this token's entries of P^T (scaled by vs).
-// Returns false, warp-uniformly, if a bounded wait ran out.
-template <int GP, bool F16P>
+// With HI_LO the S^T buffer has 32 columns: products with Q_hi in [0,16) and with Q_lo in
+// [16,32), which are added here.  Returns false, warp-uniformly, if a bounded wait ran out.
+template <int GP, bool F16P, bool HI_LO = false>
 __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j, int lane, int wq, int t,
                                                     bool valid, float sc, float vs, uint32_t tS_lane,
                                                     uint32_t tO_lane, float* red_max, uint64_t* red_bar,
                                                     uint64_t* o_ready, uint8_t* p_tile, float threshold) {
-  uint32_t sv[16];
-  tmem_ld16(tS_lane, sv);
-  tmem_wait_ld();
   float x[GP];
+  if (HI_LO) {
+    uint32_t sv[32];
+    tmem_ld32(tS_lane, sv);
+    tmem_wait_ld_regs(sv);
 #pragma unroll
-  for (int g = 0; g < GP; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
+    for (int g = 0; g < GP; ++g)
+      x[g] = valid ? (__uint_as_float(sv[g]) + __uint_as_float(sv[16 + g])) * sc : -INFINITY;
+  } else {
+    uint32_t sv[16];
+    tmem_ld16(tS_lane, sv);
+    tmem_wait_ld();
+#pragma unroll
+    for (int g = 0; g < GP; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
+  }
   float* rm = red_max + (j & 1) * 64;
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
@@ -204,16 +214,18 @@ __device__ __forceinline__ void decode_write_empty(const DecodeParams& p, int G,
   }
 }
 
-// Q^T rows of the group into the 16-row, 128B-swizzled B operand (rows >= G zero).  With f16_split,
-// Q is written as f16 hi at q_smem and f16 lo at q_smem + 4096; else as bf16 at q_smem.
+// Q^T rows of the group into the 128B-swizzled B operand, two 64-wide boxes (rows >= G zero).
+// bf16: 16 rows per box.  f16_split: 32 rows per box, f16 hi in rows [0,16) and f16 lo in rows
+// [16,32), so one N=32 MMA chain yields both partial products.
 __device__ __forceinline__ void decode_stage_q(const DecodeParams& p, int G, int kvh, int b, int wg_tid,
                                                uint8_t* q_smem, bool f16_split) {
-  constexpr int D = 128, QBOX = 16 * 128;
+  constexpr int D = 128;
+  const int box = f16_split ? 32 * 128 : 16 * 128;
   for (int c = wg_tid; c < 256; c += 128) {
     const int g = c >> 4, cc = c & 15;
     uint4 x = make_uint4(0u, 0u, 0u, 0u);
     if (g < G) x = *reinterpret_cast<const uint4*>(p.q + ((long long)b * p.Hq + (long long)kvh * G + g) * D + cc * 8);
-    const uint32_t off = (cc >> 3) * QBOX + sw128_offset(g, cc & 7);
+    const uint32_t off = (cc >> 3) * box + sw128_offset(g, cc & 7);
     if (!f16_split) {
       *reinterpret_cast<uint4*>(q_smem + off) = x;
     } else {
@@ -227,7 +239,8 @@ __device__ __forceinline__ void decode_stage_q(const DecodeParams& p, int G, int
         lo[i] = pack_f16x2(f0 - __half2float(h0), f1 - __half2float(h1));
       }
       *reinterpret_cast<uint4*>(q_smem + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(q_smem + 2 * QBOX + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * box + sw128_offset(16 + g, cc & 7)) =
+          make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
   }
 }

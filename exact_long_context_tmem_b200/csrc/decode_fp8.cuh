@@ -7,17 +7,21 @@
 //   * E4M3 -> f16 is exact (every E4M3 value is an f16 value), so the MMAs run in f16 and the
 //     fp32 scales stay out of the operands: k_scale multiplies the token's score and v_scale its
 //     probability, both on the thread that owns the token;
-//   * Q is carried as an f16 pair hi + lo (hi = f16(q), lo = f16(q - hi)) over the same K
-//     columns, so the score keeps float32-level accuracy.
+//   * Q is carried as an f16 pair hi + lo (hi = f16(q), lo = f16(q - hi)) stacked as the 32 rows of
+//     one B operand, so a single 8-step MMA chain gives both products and the score keeps
+//     float32-level accuracy.
 //
-// Roles (320 threads):
-//   warp 0      TMA producer: raw K and V code tiles through an NCS-stage ring
-//   warp 1      TMEM allocator; lane 0 issues every MMA
-//   warps 2..5  converter: thread = token; K codes -> f16 straight into TMEM (the A operand of
-//               the S MMA), V codes -> f16 in shared memory (the A operand of the PV MMA);
-//               both double-buffered so conversion runs a tile ahead of the softmax
-//   warps 6..9  softmax + epilogue: thread = token (and later = output element d)
-// TMEM columns: S^T [0,32) (two 16-column buffers), O^T [32,48), K tiles [64,128) and [128,192).
+// Roles (448 threads):
+//   warp 0       TMA producer: raw K and V code tiles through an NCS-stage ring
+//   warp 1       TMEM allocator; lane 0 issues every MMA
+//   warps 2..5   K converter: thread = token; K codes -> f16 straight into TMEM (the A operand of
+//                the S MMA), double-buffered
+//   warps 6..9   V converter: thread = token; V codes -> f16 in shared memory (the A operand of
+//                the PV MMA), double-buffered
+//   warps 10..13 softmax + epilogue: thread = token (and later = output element d)
+// The two converters run side by side and ahead of the softmax.
+// TMEM columns: S^T [0,64) (two 32-column buffers: Q_hi and Q_lo products), O^T [64,80),
+// K tiles [128,192) and [192,256).
 #pragma once
 
 #include "decode.cuh"
@@ -29,25 +33,26 @@ struct DecodeFp8Cfg {
   static constexpr int NCS = 3;                 // stages of raw code tiles
   static constexpr int CODE_TILE = 128 * 128;   // 128 tokens x 128 one-byte codes
   static constexpr int VC_TILE = 2 * 128 * 128; // 128 tokens x 128 f16, two 64-wide boxes
-  static constexpr int QBOX = 16 * 128;
-  static constexpr int Q_BYTES = 2 * QBOX;      // one of hi / lo
-  static constexpr int P_BYTES = 2 * QBOX;
+  static constexpr int QBOX = 32 * 128;         // Q_hi rows [0,16) + Q_lo rows [16,32), 64 wide
+  static constexpr int Q_BYTES = 2 * QBOX;
+  static constexpr int PBOX = 16 * 128;
+  static constexpr int P_BYTES = 2 * PBOX;
   static constexpr int OFF_KCODE = 0;
   static constexpr int OFF_VCODE = OFF_KCODE + NCS * CODE_TILE;
   static constexpr int OFF_VC = OFF_VCODE + NCS * CODE_TILE;
   static constexpr int OFF_Q = OFF_VC + 2 * VC_TILE;
-  static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_P = OFF_Q + Q_BYTES;
   static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;
   static constexpr int OFF_BAR = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;
   static constexpr int N_BARS = 4 * NCS + 1 + 2 + 2 + 1 + 8 + 1 + 2 + 1 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 448;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
 
 template <int GP>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     decode_fp8_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
   using C = DecodeFp8Cfg;
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tS0 = tmem, tO = tmem + 32, tK0 = tmem + 64;
+  const uint32_t tS0 = tmem, tO = tmem + 64, tK0 = tmem + 128;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -154,23 +159,22 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = make_idesc_f16(128, 16, false, false, false);
+      constexpr uint32_t idesc_qk = make_idesc_f16(128, 32, false, false, false);
       constexpr uint32_t idesc_pv = make_idesc_f16(128, 16, true, false, false);
       const uint32_t sQ = smem_u32(smem + C::OFF_Q);
       const uint32_t sP = smem_u32(smem + C::OFF_P);
       const uint32_t sVc = smem_u32(smem + C::OFF_VC);
-      // S^T(j) = K_j (TMEM, f16) . [Q_hi; Q_lo]^T over the same K columns
+      // S^T(j) [128 x 32] = K_j (TMEM, f16) . [Q_hi; Q_lo]^T
       auto issue_s = [&](int buf) {
-        for (int kk = 0; kk < 16; ++kk) {
-          const int kd = kk & 7;
-          const uint32_t qoff = (kk >> 3) * C::Q_BYTES + (kd >> 2) * C::QBOX + (kd & 3) * 32;
-          mma_ts(tS0 + buf * 16, tK0 + buf * 64 + kd * 8, make_sdesc_sw128(sQ + qoff, 16, 1024), idesc_qk, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t qoff = (kk >> 2) * C::QBOX + (kk & 3) * 32;
+          mma_ts(tS0 + buf * 32, tK0 + buf * 64 + kk * 8, make_sdesc_sw128(sQ + qoff, 16, 1024), idesc_qk, kk > 0);
         }
       };
       auto issue_pv = [&](int buf, bool acc) {
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t da = make_sdesc_sw128(sVc + buf * C::VC_TILE + kk * 16 * 128, 128 * 128, 1024);
-          const uint64_t db = make_sdesc_sw128(sP + buf * C::P_BYTES + (kk >> 2) * C::QBOX + (kk & 3) * 32, 16, 1024);
+          const uint64_t db = make_sdesc_sw128(sP + buf * C::P_BYTES + (kk >> 2) * C::PBOX + (kk & 3) * 32, 16, 1024);
           mma_ss(tO, da, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
@@ -217,16 +221,13 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else if (warp < 6) {
-    // ------------------------------------------------------------------ converter warpgroup
+    // ------------------------------------------------------------------ K converter warpgroup
     const int wq = warp & 3;
     const int t = wq * 32 + lane;  // token row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     ATTN_PROF_DECL(cw_k);
     ATTN_PROF_DECL(cw_kce);
     ATTN_PROF_DECL(cc_k);
-    ATTN_PROF_DECL(cw_v);
-    ATTN_PROF_DECL(cw_vce);
-    ATTN_PROF_DECL(cc_v);
     for (int j = 0; j < n; ++j) {
       const int st = j % C::NCS;
       const uint32_t ph = (j / C::NCS) & 1;
@@ -265,6 +266,24 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(&kc_full[b2]);
       ATTN_PROF_ADD(cc_k, c2);
+    }
+    if (lane == 0 && wq == 2) {
+      ATTN_PROF_FLUSH(3, cw_k);
+      ATTN_PROF_FLUSH(4, cw_kce);
+      ATTN_PROF_FLUSH(5, cc_k);
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------------ V converter warpgroup
+    const int t = (warp & 3) * 32 + lane;  // token row of the tile
+    ATTN_PROF_DECL(cw_v);
+    ATTN_PROF_DECL(cw_vce);
+    ATTN_PROF_DECL(cc_v);
+    for (int j = 0; j < n; ++j) {
+      const int st = j % C::NCS;
+      const uint32_t ph = (j / C::NCS) & 1;
+      const int b2 = j & 1;
+      const uint32_t ph2 = (j >> 1) & 1;
+      const bool valid = t0 + j * 128 + t < t1;
       // V_j -> f16 in shared memory (zeros for tokens past the length)
       ATTN_PROF_T0(c3);
       if (!mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V)) break;
@@ -279,10 +298,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&vc_full[b2]);
       ATTN_PROF_ADD(cc_v, c5);
     }
-    if (lane == 0 && wq == 2) {
-      ATTN_PROF_FLUSH(3, cw_k);
-      ATTN_PROF_FLUSH(4, cw_kce);
-      ATTN_PROF_FLUSH(5, cc_k);
+    if (lane == 0 && warp == 6) {
       ATTN_PROF_FLUSH(6, cw_v);
       ATTN_PROF_FLUSH(7, cw_vce);
       ATTN_PROF_FLUSH(8, cc_v);
@@ -292,7 +308,7 @@ __global__ void __launch_bounds__(320, 1)
     const int wq = warp & 3;
     const int t = wq * 32 + lane;  // token of the tile / TMEM lane / output element d
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int wg_tid = threadIdx.x - 192;
+    const int wg_tid = threadIdx.x - 320;
     for (int i = wg_tid; i < 2 * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
     decode_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, true);
@@ -331,9 +347,10 @@ __global__ void __launch_bounds__(320, 1)
       if (!(ok = mbar_wait_warp(&s_full[b2], ph2, SITE_DC_SM_S))) break;
       ATTN_PROF_ADD(sw_s, s1);
       tc_fence_after();
-      if (!(ok = decode_softmax_tile<GP, true>(rows, j, lane, wq, t, valid, p.scale_log2 * ks, vs,
-                                               tS0 + b2 * 16 + lane_off, tO + lane_off, red_max, red_bar, o_ready,
-                                               smem + C::OFF_P + b2 * C::P_BYTES, C::RESCALE_THRESHOLD)))
+      if (!(ok = decode_softmax_tile<GP, true, true>(rows, j, lane, wq, t, valid, p.scale_log2 * ks, vs,
+                                                     tS0 + b2 * 32 + lane_off, tO + lane_off, red_max, red_bar,
+                                                     o_ready, smem + C::OFF_P + b2 * C::P_BYTES,
+                                                     C::RESCALE_THRESHOLD)))
         break;
       fence_proxy_async_smem();
       tc_fence_before();

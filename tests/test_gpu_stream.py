@@ -82,3 +82,24 @@ def test_stream_budget_too_small(cuda_device):
     with pytest.raises(A.AttnError) as e:
         A.attn_chunked_stream(q, k, v, causal=True, chunk_tokens=512, budget_bytes=10**5)
     assert e.value.status == 4
+
+
+@pytest.mark.slow
+def test_stream_1m_tokens_sampled(cuda_device):
+    """The streamed causal prefill over 2^20 tokens (32 query / 8 KV heads, head dim 128), with
+    Q/K/V/O/LSE in pinned host memory, 64K-token key chunks and a 16e9-byte device budget,
+    checked on 64 sampled query rows (all heads) against the float64 oracle."""
+    w = I.WORKLOADS["stream_b1_h32g8_d128_s1m_chunk64k"]
+    g = I.generator(w.seed)
+    sq, skv = (w.B, w.S, w.Hq, w.D), (w.B, w.S, w.Hkv, w.D)
+    q = I.randn_bf16(sq, g, out=torch.empty(sq, dtype=torch.bfloat16, pin_memory=True))
+    k = I.randn_bf16(skv, g, out=torch.empty(skv, dtype=torch.bfloat16, pin_memory=True))
+    v = I.randn_bf16(skv, g, out=torch.empty(skv, dtype=torch.bfloat16, pin_memory=True))
+    o, lse, stats = A.attn_chunked_stream(q, k, v, causal=True, chunk_tokens=w.chunk_tokens,
+                                          budget_bytes=w.budget_bytes)
+    assert stats.plan.device_bytes <= w.budget_bytes and stats.plan.kv_chunk == w.chunk_tokens
+    rows = I.sample_rows(w.S, 60, seed=w.seed, edges=(0, 65535, 65536, w.S - 1))
+    ro, rl = O.attention(q, k, v, scale=w.scale, causal=True, rows=rows, row_chunk=64)
+    assert_o_close(o[:, rows], ro)
+    assert_lse_close(to_np(lse[:, rows]).transpose(0, 2, 1), rl)
+    device_clean()
