@@ -143,14 +143,26 @@ static int decode_splits(const attn_dims_t& d, int Tmax, int requested) {
   const int max_splits = (Tmax + 127) / 128;
   int P = requested;
   if (P <= 0) {
-    // One CTA per SM at a time (shared memory); aim for about four waves of CTAs, with every
-    // split at least 2048 tokens so the per-CTA set-up stays small next to its stream.
+    // One CTA per SM at a time (shared memory).  Take the split count, with every split at least
+    // 2048 tokens, whose CTAs fill whole waves best (at least ~4 waves, so the tail is short),
+    // preferring fewer splits on ties.
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long units = (long long)std::max(d.B, 1) * d.Hkv;
-    P = (int)std::max(1LL, (4LL * sms + units - 1) / units);
-    P = std::min(P, std::max(1, Tmax / 2048));
+    const int p_cap = std::max(1, std::min(max_splits, Tmax / 2048));
+    const int p_min = (int)std::min<long long>(p_cap, std::max(1LL, (4LL * sms + units - 1) / units));
+    double best = -1.0;
+    P = p_min;
+    for (int c = p_min; c <= std::min(p_cap, 2 * p_min + 8); ++c) {
+      const long long ctas = units * c;
+      const long long waves = (ctas + sms - 1) / sms;
+      const double fill = (double)ctas / (double)(waves * sms);
+      if (fill > best + 0.02) {
+        best = fill;
+        P = c;
+      }
+    }
   }
   P = std::min(P, max_splits);
   // Round the split length up to whole tiles, then recompute how many splits cover Tmax.
