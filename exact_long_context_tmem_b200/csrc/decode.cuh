@@ -84,11 +84,14 @@ struct DecodeRows {
 // cross-warp exchange) -> lazy O rescale -> this token's entries of P^T (scaled by vs).
 // With HI_LO the S^T buffer has 32 columns: products with Q_hi in [0,16) and with Q_lo in
 // [16,32), which are added here.  Returns false, warp-uniformly, if a bounded wait ran out.
+// prev_pv / prev_pv_parity name the barrier phase that completes when PV(j-1) has finished (the
+// O^T rescale must wait for it); the caller picks them so that the wait is unambiguous.
 template <int GP, bool F16P, bool HI_LO = false>
 __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j, int lane, int wq, int t,
                                                     bool valid, float sc, float vs, uint32_t tS_lane,
                                                     uint32_t tO_lane, float* red_max, uint64_t* red_bar,
-                                                    uint64_t* o_ready, uint8_t* p_tile, float threshold) {
+                                                    uint64_t* prev_pv, uint32_t prev_pv_parity, uint8_t* p_tile,
+                                                    float threshold) {
   float x[GP];
   if (HI_LO) {
     uint32_t sv[32];
@@ -127,7 +130,7 @@ __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j,
     }
   }
   if (need && j > 0) {  // rescale O^T row t once PV(j-1) is done
-    if (!mbar_wait_warp(o_ready, (j - 1) & 1, SITE_DC_SM_O)) return false;
+    if (!mbar_wait_warp(prev_pv, prev_pv_parity, SITE_DC_SM_O)) return false;
     tc_fence_after();
     uint32_t orow[16];
     tmem_ld16(tO_lane, orow);
@@ -447,9 +450,11 @@ __global__ void __launch_bounds__(192, 1)
       // tcgen05.ld/st are warp-collective: every lane takes the same branch around them.
       if (!(ok = mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
       tc_fence_after();
+      // PV(j-1) is the j-th completion of o_ready; S(j) completing implies PV(j-2) done, so at
+      // most one phase is pending and the parity wait is unambiguous.
       if (!(ok = decode_softmax_tile<GP, false>(rows, j, lane, wq, t, valid, p.scale_log2, 1.f,
                                                 tS0 + (j & 1) * 16 + lane_off, tO + lane_off, red_max, red_bar,
-                                                o_ready, smem + C::OFF_P + (j & 1) * C::P_BYTES,
+                                                o_ready, (j - 1) & 1, smem + C::OFF_P + (j & 1) * C::P_BYTES,
                                                 C::RESCALE_THRESHOLD)))
         break;
       if (t1 - (t0 + j * 128) < 128) {

@@ -11,17 +11,22 @@
 //     one B operand, so a single 8-step MMA chain gives both products and the score keeps
 //     float32-level accuracy.
 //
-// Roles (448 threads):
-//   warp 0       TMA producer: raw K and V code tiles through an NCS-stage ring
+// Roles (480 threads):
+//   warp 0       TMA producer of the raw K code tiles (NCS-stage ring)
+//   warp 14      TMA producer of the raw V code tiles (NCS-stage ring); a separate thread, so a
+//                V stage still waiting for its converter never holds back the next K load
 //   warp 1       TMEM allocator; lane 0 issues every MMA
 //   warps 2..5   K converter: thread = token; K codes -> f16 straight into TMEM (the A operand of
-//                the S MMA), double-buffered
+//                the S MMA)
 //   warps 6..9   V converter: thread = token; V codes -> f16 in shared memory (the A operand of
-//                the PV MMA), double-buffered
+//                the PV MMA)
 //   warps 10..13 softmax + epilogue: thread = token (and later = output element d)
-// The two converters run side by side and ahead of the softmax.
-// TMEM columns: S^T [0,64) (two 32-column buffers: Q_hi and Q_lo products), O^T [64,80),
-// K tiles [128,192) and [192,256).
+// The two converters run side by side and ahead of the softmax.  Scores, probabilities and
+// converted tiles rotate through NB = 3 buffers: S(j+3) is issued right after PV(j), so the
+// softmax has two tiles of its own work to cover the PV -> S round trip of the tensor pipe.  PV
+// completion has one barrier per buffer, so every wait on it is at most one phase behind.
+// TMEM columns: S^T [0,96) (three 32-column buffers: Q_hi and Q_lo products), O^T [96,112),
+// K tiles [128,320) (three 64-column buffers).
 #pragma once
 
 #include "decode.cuh"
@@ -31,6 +36,7 @@ namespace attn {
 struct DecodeFp8Cfg {
   static constexpr int D = 128;
   static constexpr int NCS = 3;                 // stages of raw code tiles
+  static constexpr int NB = 3;                  // S / P / converted-tile buffers
   static constexpr int CODE_TILE = 128 * 128;   // 128 tokens x 128 one-byte codes
   static constexpr int VC_TILE = 2 * 128 * 128; // 128 tokens x 128 f16, two 64-wide boxes
   static constexpr int QBOX = 32 * 128;         // Q_hi rows [0,16) + Q_lo rows [16,32), 64 wide
@@ -40,23 +46,26 @@ struct DecodeFp8Cfg {
   static constexpr int OFF_KCODE = 0;
   static constexpr int OFF_VCODE = OFF_KCODE + NCS * CODE_TILE;
   static constexpr int OFF_VC = OFF_VCODE + NCS * CODE_TILE;
-  static constexpr int OFF_Q = OFF_VC + 2 * VC_TILE;
+  static constexpr int OFF_Q = OFF_VC + NB * VC_TILE;
   static constexpr int OFF_P = OFF_Q + Q_BYTES;
-  static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_RED = OFF_P + NB * P_BYTES;
   static constexpr int OFF_BAR = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;
-  static constexpr int N_BARS = 4 * NCS + 1 + 2 + 2 + 1 + 8 + 1 + 2 + 1 + 1;
+  static constexpr int N_BARS = 4 * NCS + 1 + 7 * NB + 1 + 2 + 1 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
-  static constexpr int THREADS = 448;
-  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr int THREADS = 480;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_O = 96, COL_K = 128;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
+static_assert(DecodeFp8Cfg::SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
 template <int GP>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(480, 1)
     decode_fp8_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
   using C = DecodeFp8Cfg;
   constexpr int D = C::D;
+  constexpr int NB = C::NB;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int len = p.kv_lens[b];
@@ -70,6 +79,7 @@ __global__ void __launch_bounds__(448, 1)
     decode_write_empty(p, G, split, kvh, b);
     return;
   }
+  ATTN_PROF_T0(cta_t0);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -79,14 +89,14 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* v_full = k_empty + C::NCS;
   uint64_t* v_empty = v_full + C::NCS;
   uint64_t* q_ready = v_empty + C::NCS;
-  uint64_t* s_full = q_ready + 1;          // [2]
-  uint64_t* p_full = s_full + 2;           // [2]
-  uint64_t* o_ready = p_full + 2;
-  uint64_t* kc_full = o_ready + 1;         // [2] converted K in TMEM
-  uint64_t* kc_empty = kc_full + 2;        // [2] S MMA done reading it
-  uint64_t* vc_full = kc_empty + 2;        // [2] converted V in shared memory
-  uint64_t* vc_empty = vc_full + 2;        // [2] PV MMA done reading it
-  uint64_t* drain = vc_empty + 2;
+  uint64_t* s_full = q_ready + 1;          // [NB] S^T(j) in TMEM
+  uint64_t* p_full = s_full + NB;          // [NB] P^T(j) in shared memory
+  uint64_t* pv_done = p_full + NB;         // [NB] PV(j) completed
+  uint64_t* kc_full = pv_done + NB;        // [NB] converted K in TMEM
+  uint64_t* kc_empty = kc_full + NB;       // [NB] S MMA done reading it
+  uint64_t* vc_full = kc_empty + NB;       // [NB] converted V in shared memory
+  uint64_t* vc_empty = vc_full + NB;       // [NB] PV MMA done reading it
+  uint64_t* drain = vc_empty + NB;
   uint64_t* red_bar = drain + 1;           // [2]
   uint64_t* sum_bar = red_bar + 2;
   uint64_t* o_final = sum_bar + 1;  // single phase: every PV of the split has completed
@@ -102,16 +112,17 @@ __global__ void __launch_bounds__(448, 1)
       mbar_init(&v_empty[i], 128);
     }
     mbar_init(q_ready, 128);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NB; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
+      mbar_init(&pv_done[s], 1);
       mbar_init(&kc_full[s], 128);
       mbar_init(&kc_empty[s], 1);
       mbar_init(&vc_full[s], 128);
       mbar_init(&vc_empty[s], 1);
-      mbar_init(&red_bar[s], 128);
     }
-    mbar_init(o_ready, 1);
+    mbar_init(&red_bar[0], 128);
+    mbar_init(&red_bar[1], 128);
     mbar_init(drain, 1);
     mbar_init(sum_bar, 128);
     mbar_init(o_final, 1);
@@ -125,35 +136,29 @@ __global__ void __launch_bounds__(448, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tS0 = tmem, tO = tmem + 64, tK0 = tmem + 128;
+  const uint32_t tS0 = tmem + C::COL_S, tO = tmem + C::COL_O, tK0 = tmem + C::COL_K;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 14) {
+    // ------------------------------------------------------------------ TMA producers (K: warp 0, V: warp 14)
     if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      const bool is_k = warp == 0;
+      const CUtensorMap* tm = is_k ? &tmK : &tmV;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      uint8_t* ring = smem + (is_k ? C::OFF_KCODE : C::OFF_VCODE);
+      tma_prefetch_desc(tm);
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
         const int st = j % C::NCS;
-        const uint32_t ph = (j / C::NCS) & 1;
-        const int tok = t0 + j * 128;
-        if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, SITE_DC_LOAD_EMPTY))) break;
-        mbar_arrive_expect_tx(&k_full[st], C::CODE_TILE);
-        tma_load_4d(smem + C::OFF_KCODE + st * C::CODE_TILE, &tmK, &k_full[st], 0, kvh, tok, b);
-        issued = 2 * j + 1;
-        if (!(ok = mbar_wait(&v_empty[st], ph ^ 1, SITE_DC_LOAD_EMPTY))) break;
-        mbar_arrive_expect_tx(&v_full[st], C::CODE_TILE);
-        tma_load_4d(smem + C::OFF_VCODE + st * C::CODE_TILE, &tmV, &v_full[st], 0, kvh, tok, b);
-        issued = 2 * j + 2;
+        if (!(ok = mbar_wait(&empty[st], ((j / C::NCS) & 1) ^ 1, SITE_DC_LOAD_EMPTY))) break;
+        mbar_arrive_expect_tx(&full[st], C::CODE_TILE);
+        tma_load_4d(ring + st * C::CODE_TILE, tm, &full[st], 0, kvh, t0 + j * 128, b);
+        issued = j + 1;
       }
-      if (!ok) {
-        const int nk = (issued + 1) / 2, nv = issued / 2;
-        for (int j = (nk > C::NCS ? nk - C::NCS : 0); j < nk; ++j)
-          mbar_wait_drain(&k_full[j % C::NCS], (j / C::NCS) & 1, SITE_DC_DRAIN);
-        for (int j = (nv > C::NCS ? nv - C::NCS : 0); j < nv; ++j)
-          mbar_wait_drain(&v_full[j % C::NCS], (j / C::NCS) & 1, SITE_DC_DRAIN);
-      }
+      if (!ok)  // wait (bounded) for the copies still in flight before the CTA exits
+        for (int j = (issued > C::NCS ? issued - C::NCS : 0); j < issued; ++j)
+          mbar_wait_drain(&full[j % C::NCS], (j / C::NCS) & 1, SITE_DC_DRAIN);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(448, 1)
           mma_ts(tS0 + buf * 32, tK0 + buf * 64 + kk * 8, make_sdesc_sw128(sQ + qoff, 16, 1024), idesc_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](int buf, bool acc) {
+      auto issue_pv = [&](int buf, bool acc) {  // O^T += V_j^T . P_j^T
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t da = make_sdesc_sw128(sVc + buf * C::VC_TILE + kk * 16 * 128, 128 * 128, 1024);
           const uint64_t db = make_sdesc_sw128(sP + buf * C::P_BYTES + (kk >> 2) * C::PBOX + (kk & 3) * 32, 16, 1024);
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(448, 1)
       ATTN_PROF_DECL(pw_p);
       ATTN_PROF_DECL(pw_kc);
       bool ok = mbar_wait(q_ready, 0, SITE_DC_MMA_K);
-      for (int jj = 0; jj < 2 && jj < n && ok; ++jj) {
+      for (int jj = 0; jj < NB && jj < n && ok; ++jj) {
         if (!(ok = mbar_wait(&kc_full[jj], 0, SITE_DC_MMA_K))) break;
         tc_fence_after();
         issue_s(jj);
@@ -190,26 +195,26 @@ __global__ void __launch_bounds__(448, 1)
         mma_commit(&kc_empty[jj]);
       }
       for (int j = 0; j < n && ok; ++j) {
-        const int b2 = j & 1;
-        const uint32_t ph2 = (j >> 1) & 1;
+        const int bj = j % NB;
+        const uint32_t ph = (j / NB) & 1;
         ATTN_PROF_T0(q0);
-        if (!(ok = mbar_wait(&vc_full[b2], ph2, SITE_DC_MMA_V))) break;
+        if (!(ok = mbar_wait(&vc_full[bj], ph, SITE_DC_MMA_V))) break;
         ATTN_PROF_ADD(pw_vc, q0);
         ATTN_PROF_T0(q1);
-        if (!(ok = mbar_wait(&p_full[b2], ph2, SITE_DC_MMA_P))) break;
+        if (!(ok = mbar_wait(&p_full[bj], ph, SITE_DC_MMA_P))) break;
         ATTN_PROF_ADD(pw_p, q1);
         tc_fence_after();
-        issue_pv(b2, j > 0);
-        mma_commit(o_ready);
-        mma_commit(&vc_empty[b2]);
-        if (j + 2 < n) {
+        issue_pv(bj, j > 0);
+        mma_commit(&pv_done[bj]);
+        mma_commit(&vc_empty[bj]);
+        if (j + NB < n) {  // S(j+NB) reuses buffer bj: S(j) was read before P(j) was published
           ATTN_PROF_T0(q2);
-          if (!(ok = mbar_wait(&kc_full[b2], ((j + 2) >> 1) & 1, SITE_DC_MMA_K))) break;
+          if (!(ok = mbar_wait(&kc_full[bj], ph ^ 1, SITE_DC_MMA_K))) break;
           ATTN_PROF_ADD(pw_kc, q2);
           tc_fence_after();
-          issue_s(b2);
-          mma_commit(&s_full[b2]);
-          mma_commit(&kc_empty[b2]);
+          issue_s(bj);
+          mma_commit(&s_full[bj]);
+          mma_commit(&kc_empty[bj]);
         }
       }
       if (ok) mma_commit(o_final);
@@ -231,15 +236,15 @@ __global__ void __launch_bounds__(448, 1)
     for (int j = 0; j < n; ++j) {
       const int st = j % C::NCS;
       const uint32_t ph = (j / C::NCS) & 1;
-      const int b2 = j & 1;
-      const uint32_t ph2 = (j >> 1) & 1;
+      const int bj = j % NB;
+      const uint32_t phb = (j / NB) & 1;
       const bool valid = t0 + j * 128 + t < t1;
       // K_j -> f16 -> TMEM lane t (64 columns, two f16 per column)
       ATTN_PROF_T0(c0);
       if (!mbar_wait_warp(&k_full[st], ph, SITE_DC_SM_K)) break;
       ATTN_PROF_ADD(cw_k, c0);
       ATTN_PROF_T0(c1);
-      if (!mbar_wait_warp(&kc_empty[b2], ph2 ^ 1, SITE_DC_SM_K)) break;
+      if (!mbar_wait_warp(&kc_empty[bj], phb ^ 1, SITE_DC_SM_K)) break;  // S(j-NB) has read it
       ATTN_PROF_ADD(cw_kce, c1);
       ATTN_PROF_T0(c2);
       tc_fence_after();
@@ -259,12 +264,12 @@ __global__ void __launch_bounds__(448, 1)
             h[c4 * 8 + 2 * i + 1] = e4m3x2_to_f16x2((uint16_t)(wd[i] >> 16));
           }
         }
-        tmem_st32(tK0 + b2 * 64 + half * 32 + lane_off, h);
+        tmem_st32(tK0 + bj * 64 + half * 32 + lane_off, h);
       }
       tmem_wait_st();
       mbar_arrive(&k_empty[st]);
       tc_fence_before();
-      mbar_arrive(&kc_full[b2]);
+      mbar_arrive(&kc_full[bj]);
       ATTN_PROF_ADD(cc_k, c2);
     }
     if (lane == 0 && wq == 2) {
@@ -281,21 +286,21 @@ __global__ void __launch_bounds__(448, 1)
     for (int j = 0; j < n; ++j) {
       const int st = j % C::NCS;
       const uint32_t ph = (j / C::NCS) & 1;
-      const int b2 = j & 1;
-      const uint32_t ph2 = (j >> 1) & 1;
+      const int bj = j % NB;
+      const uint32_t phb = (j / NB) & 1;
       const bool valid = t0 + j * 128 + t < t1;
       // V_j -> f16 in shared memory (zeros for tokens past the length)
       ATTN_PROF_T0(c3);
       if (!mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V)) break;
       ATTN_PROF_ADD(cw_v, c3);
       ATTN_PROF_T0(c4);
-      if (!mbar_wait_warp(&vc_empty[b2], ph2 ^ 1, SITE_DC_SM_V)) break;
+      if (!mbar_wait_warp(&vc_empty[bj], phb ^ 1, SITE_DC_SM_V)) break;  // PV(j-NB) has read it
       ATTN_PROF_ADD(cw_vce, c4);
       ATTN_PROF_T0(c5);
-      convert_row_e4m3(smem + C::OFF_VCODE + st * C::CODE_TILE, smem + C::OFF_VC + b2 * C::VC_TILE, t, valid);
+      convert_row_e4m3(smem + C::OFF_VCODE + st * C::CODE_TILE, smem + C::OFF_VC + bj * C::VC_TILE, t, valid);
       mbar_arrive(&v_empty[st]);
       fence_proxy_async_smem();
-      mbar_arrive(&vc_full[b2]);
+      mbar_arrive(&vc_full[bj]);
       ATTN_PROF_ADD(cc_v, c5);
     }
     if (lane == 0 && warp == 6) {
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(448, 1)
     const int t = wq * 32 + lane;  // token of the tile / TMEM lane / output element d
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int wg_tid = threadIdx.x - 320;
-    for (int i = wg_tid; i < 2 * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
+    for (int i = wg_tid; i < NB * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
     decode_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, true);
     fence_proxy_async_smem();
@@ -334,8 +339,8 @@ __global__ void __launch_bounds__(448, 1)
     ATTN_PROF_DECL(sc_all);
     for (int j = 0; j < n && ok; ++j) {
       ATTN_PROF_T0(s0);
-      const int b2 = j & 1;
-      const uint32_t ph2 = (j >> 1) & 1;
+      const int bj = j % NB;
+      const uint32_t phb = (j / NB) & 1;
       const int tok = t0 + j * 128 + t;
       const bool valid = tok < t1;
       const float ks = ks_next, vs = vs_next;
@@ -344,25 +349,32 @@ __global__ void __launch_bounds__(448, 1)
         vs_next = __ldg(p.v_scale + (kv_row0 + tok + 128) * p.Hkv + kvh);
       }
       ATTN_PROF_T0(s1);
-      if (!(ok = mbar_wait_warp(&s_full[b2], ph2, SITE_DC_SM_S))) break;
+      if (!(ok = mbar_wait_warp(&s_full[bj], phb, SITE_DC_SM_S))) break;
       ATTN_PROF_ADD(sw_s, s1);
       tc_fence_after();
+      // PV(j-1) is completion number (j-1)/NB of pv_done[(j-1)%NB]; S(j) completing implies PV(j-NB)
+      // done (S(j) was issued after it), so that barrier has at most this one phase pending.
+      const int jp = j > 0 ? j - 1 : 0;
       if (!(ok = decode_softmax_tile<GP, true, true>(rows, j, lane, wq, t, valid, p.scale_log2 * ks, vs,
-                                                     tS0 + b2 * 32 + lane_off, tO + lane_off, red_max, red_bar,
-                                                     o_ready, smem + C::OFF_P + b2 * C::P_BYTES,
-                                                     C::RESCALE_THRESHOLD)))
+                                                     tS0 + bj * 32 + lane_off, tO + lane_off, red_max, red_bar,
+                                                     &pv_done[jp % NB], (uint32_t)(jp / NB) & 1,
+                                                     smem + C::OFF_P + bj * C::P_BYTES, C::RESCALE_THRESHOLD)))
         break;
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[b2]);
+      mbar_arrive(&p_full[bj]);
       ATTN_PROF_ADD(sc_all, s0);
     }
+    ATTN_PROF_T0(ep0);
+    if (ok) decode_epilogue<GP>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, o_final);
     if (lane == 0 && wq == 2) {
       ATTN_PROF_FLUSH(9, sw_s);
       ATTN_PROF_FLUSH(11, sc_all);
       ATTN_PROF_FLUSH(12, (long long)n);
+      ATTN_PROF_FLUSH(13, clock64() - ep0);
+      ATTN_PROF_FLUSH(14, ep0 - cta_t0);
+      ATTN_PROF_FLUSH(15, 1);
     }
-    if (ok) decode_epilogue<GP>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, o_final);
   }
   tc_fence_before();
   __syncthreads();
