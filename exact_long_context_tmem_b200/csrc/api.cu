@@ -186,9 +186,14 @@ static attn_status_t launch_decode_gp(const CUtensorMap& mk, const CUtensorMap& 
                                       dim3 grid, cudaStream_t stream) {
   static std::atomic<uint64_t> smem_done{0};
   if (FP8) {
-    attn_status_t st = ensure_smem(decode_fp8_sm100<GP>, DecodeFp8Cfg::SMEM_BYTES, smem_done);
+    attn_status_t st = ensure_smem(decode_fp8_sm100<GP>, DecodeFp8Cfg<GP>::SMEM_BYTES, smem_done);
     if (st != ATTN_OK) return st;
-    decode_fp8_sm100<GP><<<grid, DecodeFp8Cfg::THREADS, DecodeFp8Cfg::SMEM_BYTES, stream>>>(mk, mv, p);
+    // Persistent: one CTA per SM (at most one per work item), each walking items c, c + grid, ...
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long items = (long long)grid.x * grid.y * grid.z;
+    const dim3 pgrid((unsigned)std::min<long long>(items, std::max(sms, 1)));
+    decode_fp8_sm100<GP><<<pgrid, DecodeFp8Cfg<GP>::THREADS, DecodeFp8Cfg<GP>::SMEM_BYTES, stream>>>(mk, mv, p);
   } else {
     attn_status_t st = ensure_smem(decode_split_sm100<GP>, DecodeCfg::SMEM_BYTES, smem_done);
     if (st != ATTN_OK) return st;
@@ -230,6 +235,7 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   p.k_scale = ks;
   p.v_scale = vs;
   p.kv_lens = kv_lens;
+  p.v_codes = FP8 ? reinterpret_cast<const uint8_t*>(v) : nullptr;
   float* ws_f = reinterpret_cast<float*>(ws);
   const size_t rows = (size_t)P * d.B * d.Hq;
   p.o_part = P > 1 ? ws_f : nullptr;
@@ -237,6 +243,7 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   dim3 grid(P, d.Hkv, d.B);
+  if ((long long)P * d.Hkv * d.B > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;  // work items are int-indexed
   // The query group is padded to the next power of two (<= 16) so the kernels' per-row loops unroll.
   if (p.G <= 1) st = launch_decode_gp<FP8, 1>(mk, mv, p, grid, stream);
   else if (p.G <= 2) st = launch_decode_gp<FP8, 2>(mk, mv, p, grid, stream);
@@ -461,6 +468,11 @@ attn_status_t attn_set_wait_limit_ns(unsigned long long ns) {
 ATTN_API attn_status_t attn_debug_set_prof(void* dev_ptr) {
   unsigned long long* p = static_cast<unsigned long long*>(dev_ptr);
   ATTN_CUDA(cudaMemcpyToSymbol(g_prof, &p, sizeof(p)));
+  return ATTN_OK;
+}
+ATTN_API attn_status_t attn_debug_set_evt(void* dev_ptr) {
+  long long* p = static_cast<long long*>(dev_ptr);
+  ATTN_CUDA(cudaMemcpyToSymbol(g_evt, &p, sizeof(p)));
   return ATTN_OK;
 }
 #endif

@@ -35,6 +35,7 @@ struct DecodeParams {
   const float* k_scale;    // [B, Tmax, Hkv] (FP8) or null
   const float* v_scale;
   const int* kv_lens;       // [B]
+  const uint8_t* v_codes;   // FP8 V cache [B, Tmax, Hkv, 128] (partial tiles are copied without TMA)
   float* o_part;            // [n_splits, B, Hq, 128] when n_splits > 1
   float* lse_part;          // [n_splits, B, Hq]
   __nv_bfloat16* o;         // [B, Hq, 128] when n_splits == 1
@@ -80,33 +81,20 @@ struct DecodeRows {
 };
 
 // One tile of the decode softmax on the thread that owns token t (= TMEM lane t of S^T and, for
-// the O^T rescale, output element d = t).  Scores -> row maxima (warp redux, then a bounded
-// cross-warp exchange) -> lazy O rescale -> this token's entries of P^T (scaled by vs).
-// With HI_LO the S^T buffer has 32 columns: products with Q_hi in [0,16) and with Q_lo in
-// [16,32), which are added here.  Returns false, warp-uniformly, if a bounded wait ran out.
-// prev_pv / prev_pv_parity name the barrier phase that completes when PV(j-1) has finished (the
-// O^T rescale must wait for it); the caller picks them so that the wait is unambiguous.
-template <int GP, bool F16P, bool HI_LO = false>
-__device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j, int lane, int wq, int t,
-                                                    bool valid, float sc, float vs, uint32_t tS_lane,
+// the O^T rescale, output element d = t), from this token's scores x[g] (log2 domain, -inf for a
+// token past the length): row maxima (warp redux, then a bounded cross-warp exchange) -> lazy O
+// rescale -> this token's entries of P^T (scaled by vs).  Returns false, warp-uniformly, if a
+// bounded wait ran out.
+// j counts the tiles this warpgroup has processed (it selects the phases of red_bar); has_prev
+// says O^T already holds earlier tiles of the same split.  prev_pv / prev_pv_parity name the
+// barrier phase that completes when the previous PV has finished (the O^T rescale must wait for
+// it); the caller picks them so that the wait is unambiguous.
+template <int GP, bool F16P>
+__device__ __forceinline__ bool decode_softmax_core(DecodeRows<GP>& rows, const float (&x)[GP], int j,
+                                                    bool has_prev, int lane, int wq, int t, float vs,
                                                     uint32_t tO_lane, float* red_max, uint64_t* red_bar,
                                                     uint64_t* prev_pv, uint32_t prev_pv_parity, uint8_t* p_tile,
                                                     float threshold) {
-  float x[GP];
-  if (HI_LO) {
-    uint32_t sv[32];
-    tmem_ld32(tS_lane, sv);
-    tmem_wait_ld_regs(sv);
-#pragma unroll
-    for (int g = 0; g < GP; ++g)
-      x[g] = valid ? (__uint_as_float(sv[g]) + __uint_as_float(sv[16 + g])) * sc : -INFINITY;
-  } else {
-    uint32_t sv[16];
-    tmem_ld16(tS_lane, sv);
-    tmem_wait_ld();
-#pragma unroll
-    for (int g = 0; g < GP; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
-  }
   float* rm = red_max + (j & 1) * 64;
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
@@ -129,7 +117,7 @@ __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j,
       need = true;
     }
   }
-  if (need && j > 0) {  // rescale O^T row t once PV(j-1) is done
+  if (need && has_prev) {  // rescale O^T row t once the previous PV is done
     if (!mbar_wait_warp(prev_pv, prev_pv_parity, SITE_DC_SM_O)) return false;
     tc_fence_after();
     uint32_t orow[16];
@@ -153,14 +141,34 @@ __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j,
   return true;
 }
 
+// bf16 decode: the 16 S^T columns of this lane, scaled by sc (log2 domain), then the shared core.
+template <int GP, bool F16P>
+__device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j, bool has_prev, int lane, int wq,
+                                                    int t, bool valid, float sc, float vs, uint32_t tS_lane,
+                                                    uint32_t tO_lane, float* red_max, uint64_t* red_bar,
+                                                    uint64_t* prev_pv, uint32_t prev_pv_parity, uint8_t* p_tile,
+                                                    float threshold) {
+  uint32_t sv[16];
+  tmem_ld16(tS_lane, sv);
+  tmem_wait_ld();
+  float x[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
+  return decode_softmax_core<GP, F16P>(rows, x, j, has_prev, lane, wq, t, vs, tO_lane, red_max, red_bar, prev_pv,
+                                       prev_pv_parity, p_tile, threshold);
+}
+
 // Epilogue shared by the decode kernels: reduce the row sums over the warpgroup, wait for the last
 // PV, then thread t (= output element d) writes o[g][t] = O^T[t][g] / l_g and, for t < G, lse_t.
-// The last PV is awaited on its own single-phase barrier: on the per-tile barrier, two phases can
-// still be pending here, and a parity wait could be satisfied by the older one.
+// The last PV is awaited on a barrier that completes once per split (o_final, phase o_parity): on
+// a per-tile barrier two phases can still be pending here, and a parity wait could be satisfied
+// by the older one.  sum_parity is the phase of sum_bar; o_free (if not null) is arrived on once
+// O^T has been read, so the accumulator can take the next split.
 template <int GP>
 __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const DecodeParams& p, int G, int split,
                                                 int kvh, int b, int lane, int wq, int t, uint32_t tO_lane,
-                                                float* red_sum, uint64_t* sum_bar, uint64_t* o_final) {
+                                                float* red_sum, uint64_t* sum_bar, uint32_t sum_parity,
+                                                uint64_t* o_final, uint32_t o_parity, uint64_t* o_free) {
   constexpr int D = 128;
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
@@ -168,12 +176,16 @@ __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const Deco
     if (lane == 0) red_sum[wq * 16 + g] = s;
   }
   mbar_arrive(sum_bar);
-  if (!mbar_wait_warp(sum_bar, 0, SITE_DC_SM_S)) return false;
-  if (!mbar_wait_warp(o_final, 0, SITE_DC_SM_O)) return false;
+  if (!mbar_wait_warp(sum_bar, sum_parity, SITE_DC_SM_S)) return false;
+  if (!mbar_wait_warp(o_final, o_parity, SITE_DC_SM_O)) return false;
   tc_fence_after();
   uint32_t orow[16];
   tmem_ld16(tO_lane, orow);
   tmem_wait_ld();
+  if (o_free) {
+    tc_fence_before();
+    mbar_arrive(o_free);
+  }
   float my_lse = -INFINITY;
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
@@ -201,10 +213,11 @@ __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const Deco
   return true;
 }
 
-// Empty split: o = 0, lse = -inf (written by the whole CTA, before any barrier or TMEM use).
-__device__ __forceinline__ void decode_write_empty(const DecodeParams& p, int G, int split, int kvh, int b) {
+// Empty split: o = 0, lse = -inf, written by threads tid = 0..nthreads-1 (no barrier or TMEM use).
+__device__ __forceinline__ void decode_write_empty(const DecodeParams& p, int G, int split, int kvh, int b, int tid,
+                                                   int nthreads) {
   constexpr int D = 128;
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+  for (int i = tid; i < G * D; i += nthreads) {
     const int g = i / D, d = i % D;
     const long long h = (long long)kvh * G + g;
     if (p.n_splits == 1) {
@@ -217,34 +230,23 @@ __device__ __forceinline__ void decode_write_empty(const DecodeParams& p, int G,
   }
 }
 
-// Q^T rows of the group into the 128B-swizzled B operand, two 64-wide boxes (rows >= G zero).
-// bf16: 16 rows per box.  f16_split: 32 rows per box, f16 hi in rows [0,16) and f16 lo in rows
-// [16,32), so one N=32 MMA chain yields both partial products.
-__device__ __forceinline__ void decode_stage_q(const DecodeParams& p, int G, int kvh, int b, int wg_tid,
-                                               uint8_t* q_smem, bool f16_split) {
+// Chunk c (< 256) of the query group: row g = c / 16, elements 8 (c % 16) .. + 7 (zero for g >= G).
+__device__ __forceinline__ uint4 decode_q_chunk_load(const DecodeParams& p, int G, int kvh, int b, int c) {
   constexpr int D = 128;
-  const int box = f16_split ? 32 * 128 : 16 * 128;
-  for (int c = wg_tid; c < 256; c += 128) {
+  const int g = c >> 4, cc = c & 15;
+  uint4 x = make_uint4(0u, 0u, 0u, 0u);
+  if (g < G) x = *reinterpret_cast<const uint4*>(p.q + ((long long)b * p.Hq + (long long)kvh * G + g) * D + cc * 8);
+  return x;
+}
+
+// Q^T rows of the group into the 128B-swizzled bf16 B operand: two 64-wide boxes of 16 rows
+// (rows >= G zero).  Threads tid = 0..nthreads-1 share the work.
+__device__ __forceinline__ void decode_stage_q(const DecodeParams& p, int G, int kvh, int b, int tid, int nthreads,
+                                               uint8_t* q_smem) {
+  for (int c = tid; c < 256; c += nthreads) {
     const int g = c >> 4, cc = c & 15;
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (g < G) x = *reinterpret_cast<const uint4*>(p.q + ((long long)b * p.Hq + (long long)kvh * G + g) * D + cc * 8);
-    const uint32_t off = (cc >> 3) * box + sw128_offset(g, cc & 7);
-    if (!f16_split) {
-      *reinterpret_cast<uint4*>(q_smem + off) = x;
-    } else {
-      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float f0 = __uint_as_float(xw[i] << 16), f1 = __uint_as_float(xw[i] & 0xFFFF0000u);
-        const __half h0 = __float2half_rn(f0), h1 = __float2half_rn(f1);
-        hi[i] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-        lo[i] = pack_f16x2(f0 - __half2float(h0), f1 - __half2float(h1));
-      }
-      *reinterpret_cast<uint4*>(q_smem + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * box + sw128_offset(16 + g, cc & 7)) =
-          make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
+    *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * (16 * 128) + sw128_offset(g, cc & 7)) =
+        decode_q_chunk_load(p, G, kvh, b, c);
   }
 }
 
@@ -286,7 +288,7 @@ __global__ void __launch_bounds__(192, 1)
   const int n = t1 > t0 ? (t1 - t0 + 127) / 128 : 0;
   const int G = p.G;
   if (n == 0) {
-    decode_write_empty(p, G, split, kvh, b);
+    decode_write_empty(p, G, split, kvh, b, threadIdx.x, blockDim.x);
     return;
   }
 
@@ -432,7 +434,7 @@ __global__ void __launch_bounds__(192, 1)
     const int wg_tid = threadIdx.x - 64;
     for (int i = wg_tid; i < 2 * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
-    decode_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, false);
+    decode_stage_q(p, G, kvh, b, wg_tid, 128, smem + C::OFF_Q);
     fence_proxy_async_smem();
     mbar_arrive(q_ready);
 
@@ -452,7 +454,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       // PV(j-1) is the j-th completion of o_ready; S(j) completing implies PV(j-2) done, so at
       // most one phase is pending and the parity wait is unambiguous.
-      if (!(ok = decode_softmax_tile<GP, false>(rows, j, lane, wq, t, valid, p.scale_log2, 1.f,
+      if (!(ok = decode_softmax_tile<GP, false>(rows, j, j > 0, lane, wq, t, valid, p.scale_log2, 1.f,
                                                 tS0 + (j & 1) * 16 + lane_off, tO + lane_off, red_max, red_bar,
                                                 o_ready, (j - 1) & 1, smem + C::OFF_P + (j & 1) * C::P_BYTES,
                                                 C::RESCALE_THRESHOLD)))
@@ -472,7 +474,9 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&p_full[j & 1]);
     }
-    if (ok) decode_epilogue<GP>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, o_final);
+    if (ok)
+      decode_epilogue<GP>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, 0, o_final, 0,
+                          nullptr);
   }
   tc_fence_before();
   __syncthreads();

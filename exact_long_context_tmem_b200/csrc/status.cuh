@@ -31,6 +31,11 @@ enum WaitSite : int {
   SITE_DC_SM_V = 36,
   SITE_DC_DRAIN = 37,
   SITE_DC_SM_K = 38,
+  SITE_DC_MMA_POLL = 39,
+  SITE_DC_Q = 40,
+  SITE_DC_MMA_O = 41,
+  SITE_DC_MMA_S = 42,
+  SITE_DC_SM_P = 43,
 };
 
 // (code << 16) | site of the first error since the last reset; 0 when clean.
@@ -76,11 +81,21 @@ __device__ unsigned long long* g_prof = nullptr;
   do {                                                                \
     if (g_prof) atomicAdd(g_prof + (slot), (unsigned long long)(acc)); \
   } while (0)
+// Event timeline of CTA 0: clock64() of event `kind` (< 16) for tile `tile` (< 64).  The buffer
+// pointer is read once per thread (ATTN_EVT_INIT), so an event costs one store.
+__device__ long long* g_evt = nullptr;
+#define ATTN_EVT_INIT() long long* const evt_base_ = (blockIdx.x == 0) ? g_evt : nullptr
+#define ATTN_EVT(tile, kind)                                                      \
+  do {                                                                            \
+    if (evt_base_ && (tile) < 64) evt_base_[(tile) * 16 + (kind)] = clock64();    \
+  } while (0)
 #else
 #define ATTN_PROF_DECL(name)
 #define ATTN_PROF_T0(v)
 #define ATTN_PROF_ADD(acc, t0)
 #define ATTN_PROF_FLUSH(slot, acc)
+#define ATTN_EVT_INIT()
+#define ATTN_EVT(tile, kind)
 #endif
 
 }  // namespace attn

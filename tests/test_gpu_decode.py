@@ -50,7 +50,7 @@ def test_decode_bf16_ragged_with_nan_padding(cuda_device, splits):
     device_clean()
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (16, 16), (12, 1), (6, 3)])
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (16, 16), (12, 1), (6, 3), (64, 8), (32, 2)])
 def test_decode_bf16_groups(cuda_device, Hq, Hkv):
     w, d = _small(2, Hq, Hkv, [1, 2049], 2100, seed=Hq * 10 + Hkv)
     for splits in (1, 5):
@@ -68,6 +68,52 @@ def test_decode_fp8_small(cuda_device, splits):
     ro, rl = _ref(d, w.scale, fp8=True)
     assert_o_close(o, ro)
     assert_lse_close(lse, rl)
+    device_clean()
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (16, 16), (12, 1), (6, 3), (64, 8), (32, 2)])
+def test_decode_fp8_groups(cuda_device, Hq, Hkv):
+    w, d = _small(2, Hq, Hkv, [1, 2049], 2100, seed=Hq * 10 + Hkv + 500, fp8=True)
+    for splits in (1, 5):
+        o, lse = _run(d, cuda_device, splits, fp8=True)
+        ro, rl = _ref(d, w.scale, fp8=True)
+        assert_o_close(o, ro)
+        assert_lse_close(lse, rl)
+    device_clean()
+
+
+def test_decode_fp8_many_items_ragged(cuda_device):
+    """More (split, head, sequence) items than SMs: each persistent CTA runs several items back to
+    back, with empty, one-token and exact-tile splits among them."""
+    g = np.random.default_rng(77)
+    lens = g.integers(0, 1501, size=40)
+    lens[:6] = [0, 1, 1500, 128, 129, 0]
+    w, d = _small(40, 8, 2, lens.tolist(), 1500, seed=77, fp8=True)
+    for splits in (4, 1):
+        o, lse = _run(d, cuda_device, splits, fp8=True)
+        ro, rl = _ref(d, w.scale, fp8=True)
+        assert_o_close(o, ro)
+        assert_lse_close(lse, rl)
+        assert torch.all(o[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    device_clean()
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_decode_rescale_ramp(cuda_device, fp8):
+    """Key magnitudes grow along the sequence, so the running maximum rises by more than the lazy
+    threshold on almost every tile and O^T is rescaled again and again."""
+    Tmax = 2000
+    w, d = _small(2, 32, 8, [2000, 1700], Tmax, seed=91, fp8=fp8)
+    ramp = 1.0 + torch.arange(Tmax, dtype=torch.float32) / 32.0
+    if fp8:
+        d["k_scale"] = d["k_scale"] * ramp[None, :, None]
+    else:
+        d["k"] = (d["k"].float() * ramp[None, :, None, None]).to(torch.bfloat16)
+    for splits in (1, 3):
+        o, lse = _run(d, cuda_device, splits, fp8=fp8)
+        ro, rl = _ref(d, w.scale, fp8=fp8)
+        assert_o_close(o, ro)
+        assert_lse_close(lse, rl)
     device_clean()
 
 
