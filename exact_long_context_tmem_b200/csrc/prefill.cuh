@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   if (threadIdx.x == 0) ATTN_TRACE_AT(0, 3, n);
+  ATTN_EVT_INIT();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -233,8 +234,10 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait(&k_full[0], 0, SITE_PF_MMA_K);
         if (ok) {
           tc_fence_after();
+          ATTN_EVT(0, 0);
           issue_qk(0, 0);
           mma_commit(&s_full[0]);
+          ATTN_EVT(0, 8);
           issue_qk(1, 0);
           mma_commit(&s_full[1]);
           mma_commit(&k_empty[0]);
@@ -252,10 +255,12 @@ __global__ void __launch_bounds__(384, 1)
         if (!(ok = mbar_wait(&p_full[0], j & 1, SITE_PF_MMA_P))) break;
         ATTN_TRACE_AT(1, 7, j);
         tc_fence_after();
+        ATTN_EVT(j, 3);
         issue_pv(0, st, j > 0);
         if (more) {
           if (!(ok = mbar_wait(&k_full[st1], ph1, SITE_PF_MMA_K))) break;
           tc_fence_after();
+          ATTN_EVT(j + 1, 0);
           issue_qk(0, st1);
           mma_commit(&s_full[0]);
         }
@@ -263,9 +268,11 @@ __global__ void __launch_bounds__(384, 1)
         if (!(ok = mbar_wait(&p_full[1], j & 1, SITE_PF_MMA_P))) break;
         ATTN_TRACE_AT(1, 9, j);
         tc_fence_after();
+        ATTN_EVT(j, 11);
         issue_pv(1, st, j > 0);
         mma_commit(&v_empty[st]);
         if (more) {
+          ATTN_EVT(j + 1, 8);
           issue_qk(1, st1);
           mma_commit(&s_full[1]);
           mma_commit(&k_empty[st1]);
@@ -296,6 +303,7 @@ __global__ void __launch_bounds__(384, 1)
       // tcgen05.ld/st are warp-collective: every lane takes the same branch around them.
       if (!(ok = mbar_wait_warp(&s_full[slot], j & 1, SITE_PF_SM_S))) break;
       if (r == 0) ATTN_TRACE_AT(2 + slot, 2, j);
+      if (r == 0) ATTN_EVT(j, slot * 8 + 1);
       tc_fence_after();
       const int kv0 = j * 128;
       long long lim64 = (long long)p.T - kv0;  // column c is a visible key iff c < lim
@@ -345,6 +353,7 @@ __global__ void __launch_bounds__(384, 1)
           tmem_wait_st();
         }
       }
+      if (r == 0) ATTN_EVT(j, slot * 8 + 2);
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
       // p = 2^(s * scale * log2 e - m) in packed fp32 pairs; one pair in ATTN_PREFILL_POLY_PERIOD
       // goes to the FMA pipe (polynomial) and the rest to the MUFU.  P is stored per 32 scores (16 packed columns, over
@@ -366,9 +375,9 @@ __global__ void __launch_bounds__(384, 1)
             e.x = ex2_approx(x.x);
             e.y = ex2_approx(x.y);
           }
+          pk[i] = pack_bf16x2(e.x, e.y);
           if (i & 1) acc1 = add2(acc1, e);
           else acc0 = add2(acc0, e);
-          pk[i] = pack_bf16x2(e.x, e.y);
         }
         tmem_st16(tS + c * 16, pk);
       }
@@ -378,6 +387,7 @@ __global__ void __launch_bounds__(384, 1)
       if (r == 0) ATTN_TRACE_AT(2 + slot, 4, j);
       tc_fence_before();
       mbar_arrive(&p_full[slot]);
+      if (r == 0) ATTN_EVT(j, slot * 8 + 4);
     }
     // ---- epilogue: O / l -> global, LSE = ln2 * (m + log2 l)
     const int row = q_lo + r;
