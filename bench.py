@@ -284,12 +284,22 @@ def bench_prefill(w, steps, warmup, world, dev, pk):
     }
 
 
-def bench_decode(name, steps, warmup, world, dev, pk):
+PAGE_SIZE = 512
+
+
+def bench_decode(name, steps, warmup, world, dev, pk, paged=False):
+    """Split-KV decode of a decode workload; paged=True lays the same cache out as a pool of
+    PAGE_SIZE-token pages in seeded random order with a page table (attn_decode_paged)."""
     from exact_long_context_tmem_b200 import attn as A
 
     w = I.WORKLOADS[name]
     d = I.decode_inputs(w)
     lens = d["kv_lens"]
+    Tmax = d["Tmax"]
+    if paged:
+        d = I.paged_inputs(d, PAGE_SIZE, seed=w.seed + 7)
+        Tmax = d["page_table"].shape[1] * PAGE_SIZE
+        table = d["page_table"].to(dev)
     qd, ld = d["q"].to(dev), lens.to(dev)
     if w.kv_fp8:
         kd, vd = d["k_codes"].to(dev), d["v_codes"].to(dev)
@@ -297,7 +307,6 @@ def bench_decode(name, steps, warmup, world, dev, pk):
     else:
         kd, vd = d["k"].to(dev), d["v"].to(dev)
         ks = vs = None
-    Tmax = d["Tmax"]
     o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
     nbytes = A.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, Tmax)
@@ -305,7 +314,10 @@ def bench_decode(name, steps, warmup, world, dev, pk):
     splits = A.attn_decode_num_splits(w.B, w.Hq, w.Hkv, w.D, Tmax)
 
     def step():
-        A.attn_decode_splitkv(qd, kd, vd, ld, k_scale=ks, v_scale=vs, o=o, lse=lse, ws=ws)
+        if paged:
+            A.attn_decode_paged(qd, kd, vd, table, ld, k_scale=ks, v_scale=vs, o=o, lse=lse, ws=ws)
+        else:
+            A.attn_decode_splitkv(qd, kd, vd, ld, k_scale=ks, v_scale=vs, o=o, lse=lse, ws=ws)
 
     for _ in range(warmup):
         step()
@@ -321,10 +333,11 @@ def bench_decode(name, steps, warmup, world, dev, pk):
     call_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
     nb = decode_bytes(w, lens)
     gbs = nb / (call_ms * 1e-3) / 1e9
-    return {"workload": name, "value": round(gbs * world, 1), "unit": "GB/s", "ms_per_step": round(call_ms, 4),
+    return {"workload": name + (f"_paged{PAGE_SIZE}" if paged else ""), "value": round(gbs * world, 1), "unit": "GB/s",
+            "ms_per_step": round(call_ms, 4),
             "splits": splits, "kv_tokens": int(lens.sum()), "bytes_per_step": nb,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": ncu_traffic(name),
+                         "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": None if paged else ncu_traffic(name),
                          "timed": "split kernel + merge kernel (one API call)"},
             "launches": steps * (2 if splits > 1 else 1)}
 
@@ -388,7 +401,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--stream", action="store_true", help="also run the 1M-token streamed prefill")
     ap.add_argument("--cpu-rows", type=int, default=128)
-    ap.add_argument("--workloads", default="prefill,decode_bf16,decode_fp8",
+    ap.add_argument("--workloads", default="prefill,decode_bf16,decode_fp8,decode_bf16_paged,decode_fp8_paged",
                     help="comma list of prefill, decode_bf16, decode_fp8 (profiling runs select one)")
     args = ap.parse_args()
     w = I.WORKLOADS[HEADLINE]
@@ -435,6 +448,8 @@ def main():
         for key, name in zip(("decode_bf16", "decode_fp8"), DECODE_WORKLOADS):
             if key in sel:
                 dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk))
+            if key + "_paged" in sel:
+                dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk, paged=True))
     st, site = A.attn_device_status(reset=True)
     if st != 0:
         raise SystemExit(f"device status {st} at wait site {site}")

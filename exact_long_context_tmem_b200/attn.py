@@ -17,13 +17,15 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libattn.so")
 
 ATTN_OK = 0
+ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA = 1, 2, 3
+ATTN_ERR_BUDGET, ATTN_ERR_TIMEOUT, ATTN_ERR_INJECTED = 4, 5, 6
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "budget", 5: "timeout",
           6: "injected"}
 ATTN_BF16, ATTN_FP8_E4M3, ATTN_F32 = 0, 1, 2
 
 EXPORTS = [
     "attn_prefill", "attn_decode_workspace_bytes", "attn_decode_num_splits", "attn_decode_splitkv",
-    "attn_decode_splitkv_noalloc",
+    "attn_decode_splitkv_noalloc", "attn_decode_paged",
     "attn_merge_lse", "attn_stream_plan", "attn_stream_task", "attn_chunked_stream", "attn_status_string",
     "attn_last_cuda_error", "attn_device_status", "attn_set_wait_limit_ns", "attn_debug_wait_probe",
     "attn_debug_inject", "attn_debug_exp2",
@@ -73,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.attn_decode_splitkv.restype = i
     L.attn_decode_splitkv_noalloc.argtypes = [vp, vp, vp, i, vp, vp, vp, i, Dims, i, vp, vp, vp]
     L.attn_decode_splitkv_noalloc.restype = i
+    L.attn_decode_paged.argtypes = [vp, vp, vp, i, vp, vp, vp, i, i, i, vp, Dims, i, vp, vp, vp, sz, vp]
+    L.attn_decode_paged.restype = i
     L.attn_merge_lse.argtypes = [vp, vp, i, ll, i, vp, i, vp, i, vp]
     L.attn_merge_lse.restype = i
     L.attn_stream_plan.argtypes = [Dims, ll, i, ll, sz, ctypes.POINTER(StreamPlan)]
@@ -175,6 +179,35 @@ def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: 
                                    _ptr(v_scale), _ptr(kv_lens), int(Tmax), dims, int(num_splits), _ptr(o),
                                    _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_decode_paged(q, k_pool, v_pool, page_table, kv_lens, *, k_scale=None, v_scale=None,
+                      scale: float | None = None, num_splits: int = 0, o=None, lse=None, ws=None,
+                      want_lse: bool = True, stream=None):
+    """q [B,Hq,D] bf16; k_pool/v_pool [num_pages, page_size, Hkv, D] bf16 or uint8 E4M3 codes
+    (+ float32 scale pools [num_pages, page_size, Hkv]); page_table int32 [B, max_pages] and
+    kv_lens int32 [B] on the device -> (o [B,Hq,D] bf16, lse [B,Hq] float32)."""
+    _need_cuda(q, k_pool, v_pool, page_table, kv_lens, k_scale, v_scale)
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv = k_pool.shape[0], k_pool.shape[1], k_pool.shape[2]
+    max_pages = page_table.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    fp8 = k_pool.dtype in (torch.uint8, torch.float8_e4m3fn)
+    dims = _dims(B, Hq, Hkv, D, scale)
+    if o is None:
+        o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = int(lib().attn_decode_workspace_bytes(dims, int(max_pages * page_size), int(num_splits)))
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().attn_decode_paged(_ptr(q), _ptr(k_pool), _ptr(v_pool), ATTN_FP8_E4M3 if fp8 else ATTN_BF16,
+                                 _ptr(k_scale), _ptr(v_scale), _ptr(page_table), int(max_pages), int(page_size),
+                                 int(num_pages), _ptr(kv_lens), dims, int(num_splits), _ptr(o), _ptr(lse), _ptr(ws),
+                                 ws_bytes, _stream(stream))
+    _check(st, "attn_decode_paged")
     return o, lse
 
 

@@ -203,14 +203,21 @@ static attn_status_t launch_decode_gp(const CUtensorMap& mk, const CUtensorMap& 
   return ATTN_OK;
 }
 
+// Where the cache lives: a padded [B, Tmax] cache is the page table-free case (one page of Tmax
+// tokens per sequence); a paged pool is [num_pages, page_size] with a device page table.
+struct DecodePaging {
+  const int* table;
+  int max_pages, page_size, num_pages;
+};
+
 template <bool FP8>
 static attn_status_t launch_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
                                    const int* kv_lens, int Tmax, const attn_dims_t& d, int P, int split_tokens,
-                                   void* o, float* lse, void* ws, cudaStream_t stream) {
+                                   void* o, float* lse, void* ws, cudaStream_t stream, const DecodePaging& pg) {
   attn_status_t st;
   CUtensorMap mk, mv;
   // With Tmax == 0 every split is empty and no map is read; it still needs a valid base and extent.
-  const uint64_t dk[4] = {128, (uint64_t)d.Hkv, (uint64_t)std::max(Tmax, 1), (uint64_t)d.B};
+  const uint64_t dk[4] = {128, (uint64_t)d.Hkv, (uint64_t)std::max(pg.page_size, 1), (uint64_t)std::max(pg.num_pages, 1)};
   const void* kb = Tmax > 0 ? k : q;
   const void* vb = Tmax > 0 ? v : q;
   if (FP8) {
@@ -236,6 +243,10 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   p.v_scale = vs;
   p.kv_lens = kv_lens;
   p.v_codes = FP8 ? reinterpret_cast<const uint8_t*>(v) : nullptr;
+  p.page_table = pg.table;
+  p.max_pages = pg.max_pages;
+  p.page_size = std::max(pg.page_size, 1);
+  p.num_pages = pg.num_pages;
   float* ws_f = reinterpret_cast<float*>(ws);
   const size_t rows = (size_t)P * d.B * d.Hq;
   p.o_part = P > 1 ? ws_f : nullptr;
@@ -380,8 +391,41 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, a
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int per = decode_split_tokens(Tmax, P);
-  if (fp8) return launch_decode<true>(q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st);
-  return launch_decode<false>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st);
+  const DecodePaging pg{nullptr, 1, Tmax, dims.B};
+  if (fp8) return launch_decode<true>(q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
+  return launch_decode<false>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, attn_dtype_t kv_dtype,
+                                const float* k_scale_pool, const float* v_scale_pool, const int* page_table,
+                                int max_pages, int page_size, int num_pages, const int* kv_lens, attn_dims_t dims,
+                                int num_splits, void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!dims_ok(dims) || num_splits < 0 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
+  if (kv_dtype != ATTN_BF16 && kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (max_pages < 1 || page_size < 128 || page_size % 128 != 0 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+  if ((long long)max_pages * page_size > 0x7fffffffLL || (long long)num_pages * page_size > 0x7fffffffLL)
+    return ATTN_ERR_UNSUPPORTED;
+  if (dims.B == 0) return ATTN_OK;
+  if (!q || !o || !kv_lens || !page_table || !k_pool || !v_pool) return ATTN_ERR_INVALID_ARG;
+  const bool fp8 = kv_dtype == ATTN_FP8_E4M3;
+  if (fp8 != (k_scale_pool != nullptr) || fp8 != (v_scale_pool != nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned4(kv_lens) || !aligned4(page_table) || (lse && !aligned4(lse)))
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool)) return ATTN_ERR_INVALID_ARG;
+  if (fp8 && (!aligned4(k_scale_pool) || !aligned4(v_scale_pool))) return ATTN_ERR_INVALID_ARG;
+  if (dims.D != 128 || dims.Hq / dims.Hkv > 16) return ATTN_ERR_UNSUPPORTED;
+  if (dims.B > 65535 || dims.Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  const int Tmax = max_pages * page_size;
+  const int P = decode_splits(dims, Tmax, num_splits);
+  const size_t need = decode_ws_bytes(dims, P);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int per = decode_split_tokens(Tmax, P);
+  const DecodePaging pg{page_table, max_pages, page_size, num_pages};
+  if (fp8)
+    return launch_decode<true>(q, k_pool, v_pool, k_scale_pool, v_scale_pool, kv_lens, Tmax, dims, P, per, o, lse, ws,
+                               st, pg);
+  return launch_decode<false>(q, k_pool, v_pool, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
 }
 
 // Split-KV decode without allocation: the split partials live in this static device array
@@ -453,7 +497,9 @@ attn_status_t attn_device_status(int reset, int* site) {
   }
   if (site) *site = (int)(v & 0xFFFFu);
   if (v == 0) return ATTN_OK;
-  return ((v >> 16) == ATTN_DEV_TIMEOUT) ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
+  if ((v >> 16) == ATTN_DEV_TIMEOUT) return ATTN_ERR_TIMEOUT;
+  if ((v >> 16) == ATTN_DEV_BAD_PAGE) return ATTN_ERR_INVALID_ARG;
+  return ATTN_ERR_CUDA;
 }
 
 attn_status_t attn_set_wait_limit_ns(unsigned long long ns) {

@@ -35,11 +35,48 @@ struct DecodeParams {
   const float* k_scale;    // [B, Tmax, Hkv] (FP8) or null
   const float* v_scale;
   const int* kv_lens;       // [B]
-  const uint8_t* v_codes;   // FP8 V cache [B, Tmax, Hkv, 128] (partial tiles are copied without TMA)
+  const uint8_t* v_codes;   // FP8 V pool [num_pages, page_size, Hkv, 128] (partial tiles are copied without TMA)
+  // Paged cache (LLM-CoOpt summary, "Opt-Pa"): token t of sequence b lives in pool page
+  // page_table[b * max_pages + t / page_size] at offset t % page_size.  Without a table the cache
+  // is one page of Tmax tokens per sequence (page_size = Tmax, num_pages = B, page of b = b).
+  const int* page_table;    // device int32 [B, max_pages] or null
+  int max_pages, page_size, num_pages;
   float* o_part;            // [n_splits, B, Hq, 128] when n_splits > 1
   float* lse_part;          // [n_splits, B, Hq]
   __nv_bfloat16* o;         // [B, Hq, 128] when n_splits == 1
   float* lse;               // [B, Hq] or null
+};
+
+// Pool page of the tile of sequence b that starts at token tok (a multiple of 128; with a table,
+// page_size is a multiple of 128, so a tile never straddles two pages).  Table entries are read
+// one page ahead of their use, so the load latency stays off the copy issue; an entry outside
+// [0, num_pages) is reported through the device status word and gives page -1, which the callers
+// never dereference (a TMA box at page -1 lands as zeros).
+struct PageCursor {
+  int b = -1, lp = -1, page = 0;  // the page in use
+  int nb = -1, nlp = -1, nraw = 0;  // the next page of the same sequence, loaded ahead
+  __device__ __forceinline__ int offset(const DecodeParams& p, int tok) const {
+    return p.page_table ? tok % p.page_size : tok;
+  }
+  __device__ __forceinline__ int get(const DecodeParams& p, int b_, int tok) {
+    if (!p.page_table) return b_;
+    const int l = tok / p.page_size;
+    if (b_ == b && l == lp) return page;
+    int raw;
+    if (b_ == nb && l == nlp) raw = nraw;
+    else raw = __ldg(p.page_table + (long long)b_ * p.max_pages + l);
+    if (raw < 0 || raw >= p.num_pages) {
+      record_device_error(ATTN_DEV_BAD_PAGE, SITE_DC_PAGE);
+      raw = -1;
+    }
+    b = b_;
+    lp = l;
+    page = raw;
+    nb = b_;
+    nlp = l + 1;
+    nraw = nlp < p.max_pages ? __ldg(p.page_table + (long long)b_ * p.max_pages + nlp) : -1;
+    return page;
+  }
 };
 
 struct DecodeCfg {
@@ -347,19 +384,21 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch_desc(&tmV);
       int issued = 0;
       bool ok = true;
+      PageCursor pc;
       for (int j = 0; j < n; ++j) {
         const int st = j % C::NST;
         const uint32_t ph = (j / C::NST) & 1;
         const int tok = t0 + j * 128;
+        const int pg = pc.get(p, b, tok), off = pc.offset(p, tok);
         if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, SITE_DC_LOAD_EMPTY))) break;
         mbar_arrive_expect_tx(&k_full[st], C::KV_TILE);
-        tma_load_4d(smem + C::OFF_K + st * C::KV_TILE, &tmK, &k_full[st], 0, kvh, tok, b);
-        tma_load_4d(smem + C::OFF_K + st * C::KV_TILE + 128 * 128, &tmK, &k_full[st], 64, kvh, tok, b);
+        tma_load_4d(smem + C::OFF_K + st * C::KV_TILE, &tmK, &k_full[st], 0, kvh, off, pg);
+        tma_load_4d(smem + C::OFF_K + st * C::KV_TILE + 128 * 128, &tmK, &k_full[st], 64, kvh, off, pg);
         issued = 2 * j + 1;
         if (!(ok = mbar_wait(&v_empty[st], ph ^ 1, SITE_DC_LOAD_EMPTY))) break;
         mbar_arrive_expect_tx(&v_full[st], C::KV_TILE);
-        tma_load_4d(smem + C::OFF_V + st * C::KV_TILE, &tmV, &v_full[st], 0, kvh, tok, b);
-        tma_load_4d(smem + C::OFF_V + st * C::KV_TILE + 128 * 128, &tmV, &v_full[st], 64, kvh, tok, b);
+        tma_load_4d(smem + C::OFF_V + st * C::KV_TILE, &tmV, &v_full[st], 0, kvh, off, pg);
+        tma_load_4d(smem + C::OFF_V + st * C::KV_TILE + 128 * 128, &tmV, &v_full[st], 64, kvh, off, pg);
         issued = 2 * j + 2;
       }
       if (!ok) {

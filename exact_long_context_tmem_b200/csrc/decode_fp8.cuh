@@ -68,8 +68,9 @@ struct DecodeFp8Cfg {
   static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_QEXP = OFF_P + NS * P_BYTES;  // [2][16] row exponents e
   static constexpr int OFF_RED = OFF_QEXP + 2 * 16 * 4;
-  static constexpr int OFF_BAR = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;
-  static constexpr int N_BARS = NCS_K + 4 * NS + 10 + 4;
+  static constexpr int OFF_SCALE = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;  // [NCS_V][k, v][128] per-token scales
+  static constexpr int OFF_BAR = OFF_SCALE + NCS_V * 2 * 128 * 4;
+  static constexpr int N_BARS = NCS_K + 4 * NS + 10 + 4 + NCS_V;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
   static constexpr int THREADS = 256;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -116,32 +117,6 @@ struct DecodeItemIter {
       if (cur.n > 0) return true;
     }
     return false;
-  }
-};
-
-// Walks the same tile sequence as DecodeItemIter (tiles of this CTA's non-empty items) for the
-// softmax's per-token scale loads, which run several tiles ahead of their use: under a full HBM
-// load a global load takes microseconds.
-struct ScaleCursor {
-  DecodeItemIter it;
-  int l = 0;
-  bool valid;
-  __device__ __forceinline__ explicit ScaleCursor(const DecodeParams& p) : it(p) { valid = it.next(p); }
-  __device__ __forceinline__ void load(const DecodeParams& p, int t, float& ks, float& vs) const {
-    ks = 1.f;
-    vs = 1.f;
-    const int tok = it.cur.t0 + l * 128 + t;
-    if (valid && tok < it.cur.t1) {
-      const long long r = ((long long)it.cur.b * p.Tmax + tok) * p.Hkv + it.cur.kvh;
-      ks = __ldg(p.k_scale + r);
-      vs = __ldg(p.v_scale + r);
-    }
-  }
-  __device__ __forceinline__ void advance(const DecodeParams& p) {
-    if (valid && ++l == it.cur.n) {
-      l = 0;
-      valid = it.next(p);
-    }
   }
 };
 
@@ -418,7 +393,9 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* drain = sum_bar + 1;       // S issuer's MMAs completed
   uint64_t* drain_pv = drain + 1;      // PV issuer's MMAs completed
   uint64_t* exp_bar = drain_pv + 1;    // the softmax's row exponents of an item are in q_exp
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(exp_bar + 1);
+  uint64_t* sc_full = exp_bar + 1;     // [NCS_V] the per-token scales of V stage j % NCS_V landed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sc_full + NCS_V);
+  float* scales = reinterpret_cast<float*>(smem + C::OFF_SCALE);  // [NCS_V][2][128]
   int* q_exp = reinterpret_cast<int*>(smem + C::OFF_QEXP);       // [2][16] softmax's row exponents
   float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][16]
   float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
@@ -442,6 +419,7 @@ __global__ void __launch_bounds__(256, 1)
     mbar_init(drain, 1);
     mbar_init(drain_pv, 1);
     mbar_init(exp_bar, 128);
+    for (int i = 0; i < NCS_V; ++i) mbar_init(&sc_full[i], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -468,9 +446,12 @@ __global__ void __launch_bounds__(256, 1)
       DecodeItemIter it(p);
       int j = 0;  // tiles issued
       bool ok = true;
+      PageCursor pc;
       while (ok && it.next(p)) {
         for (int l = 0; l < it.cur.n; ++l, ++j) {
           const int st = j % NCS_K;
+          const int tok0 = it.cur.t0 + l * 128;
+          const int pg = pc.get(p, it.cur.b, tok0);
           // Stage st last held tile j - NCS_K: S(j - NCS_K) completing frees it.  That barrier phase
           // is unambiguous: S(j - NCS_K - NS) completed before tile j - NS was loaded, and the next
           // S on the barrier, S(j - NCS_K + NS), needs a later load (NS > NCS_K).
@@ -479,7 +460,7 @@ __global__ void __launch_bounds__(256, 1)
           mbar_arrive_expect_tx(&k_full[st], C::CODE_TILE);
           ATTN_EVT(j, 0);
           tma_load_4d(smem + C::OFF_KCODE + st * C::CODE_TILE, &tmK, &k_full[st], 0, it.cur.kvh,
-                      it.cur.t0 + l * 128, it.cur.b);
+                      pc.offset(p, tok0), pg);
         }
       }
       if (!ok)  // wait (bounded) for the copies still in flight before the CTA exits
@@ -501,6 +482,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     int j = 0, ie = 0;
     bool ok = true;
+    PageCursor vpc;
     while (ok && it.next(p)) {
       const int qb = ie & 1;
       if (!(ok = mbar_wait_warp(&q_free[qb], ((ie >> 1) & 1) ^ 1, SITE_DC_Q))) break;
@@ -543,19 +525,38 @@ __global__ void __launch_bounds__(256, 1)
           break;
         uint8_t* dst = smem + C::OFF_VCODE + st * C::CODE_TILE;
         const int tok0 = it.cur.t0 + l * 128;
+        const int pg = vpc.get(p, it.cur.b, tok0), off = vpc.offset(p, tok0);
+        {
+          // The tile's k and v scales go into the scale stage with the codes, so the softmax reads
+          // them from shared memory (no global load, no page lookup on its path).  Tokens past the
+          // split (or on an invalid page) get 0, which their masked scores never use.
+          const long long base = ((long long)(pg >= 0 ? pg : 0) * p.page_size + off) * p.Hkv + it.cur.kvh;
+          float* sdst = scales + st * 256;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int i = lane + 32 * m, tk = i & 127;
+            const bool in = pg >= 0 && tok0 + tk < it.cur.t1;
+            const float* src = (i < 128 ? p.k_scale : p.v_scale) + (in ? base + (long long)tk * p.Hkv : 0);
+            cp_async_4_zfill(sdst + i, src, in ? 4u : 0u);
+          }
+          cp_async_mbar_arrive(&sc_full[st]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sc_full[st]);
+        }
         if (tok0 + 128 <= it.cur.t1) {
           if (lane == 0) {
             mbar_arrive_expect_tx(&p_full[j % NS], C::CODE_TILE);
             ATTN_EVT(j, 8);
-            tma_load_4d(dst, &tmV, &p_full[j % NS], 0, it.cur.kvh, tok0, it.cur.b);
+            tma_load_4d(dst, &tmV, &p_full[j % NS], 0, it.cur.kvh, off, pg);
           }
         } else {
           // The split's last, partial tile: the PV MMA reads the codes as they are, and cache
           // slots past the length may hold anything (NaN codes included), so the tile comes in
           // through zero-filling 16-byte copies laid out like the TMA's 128-byte swizzle.
-          const int nvalid = it.cur.t1 - tok0;
+          // (an invalid page, already reported, reads nothing: every row is zero-filled)
+          const int nvalid = pg >= 0 ? it.cur.t1 - tok0 : 0;
           const uint8_t* src = reinterpret_cast<const uint8_t*>(p.v_codes) +
-                               (((long long)it.cur.b * p.Tmax + tok0) * p.Hkv + it.cur.kvh) * 128;
+                               (((long long)(pg >= 0 ? pg : 0) * p.page_size + off) * p.Hkv + it.cur.kvh) * 128;
 #pragma unroll 4
           for (int i = 0; i < 32; ++i) {
             const int c = lane + 32 * i, r = c >> 3, ch = c & 7;
@@ -665,15 +666,6 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int wg_tid = threadIdx.x - 96;  // warps 3..6
     const int n_items = p.n_splits * p.Hkv * p.B;
-    // Per-token scales, SCALE_AHEAD tiles ahead of their use (queue shifted once per tile).
-    constexpr int SCALE_AHEAD = 4;
-    ScaleCursor scur(p);
-    float ksq[SCALE_AHEAD], vsq[SCALE_AHEAD];
-#pragma unroll
-    for (int r = 0; r < SCALE_AHEAD; ++r) {
-      scur.load(p, t, ksq[r], vsq[r]);
-      scur.advance(p);
-    }
     // The row exponents e are recomputed here (the same function of the same bf16 query as the Q
     // stager's): thread wg_tid takes elements 16 (wg_tid % 8) .. + 15 of row wg_tid / 8, loaded
     // one item ahead, and the row maxima meet in shared memory.
@@ -726,14 +718,11 @@ __global__ void __launch_bounds__(256, 1)
       for (int l = 0; l < cur.n; ++l, ++j) {
         const int bs = j % NS;
         const bool valid = cur.t0 + l * 128 + t < cur.t1;
-        const float ks = ksq[0], vs = vsq[0];
-#pragma unroll
-        for (int r = 0; r + 1 < SCALE_AHEAD; ++r) {
-          ksq[r] = ksq[r + 1];
-          vsq[r] = vsq[r + 1];
-        }
-        scur.load(p, t, ksq[SCALE_AHEAD - 1], vsq[SCALE_AHEAD - 1]);
-        scur.advance(p);
+        // scales of tile j: staged with V(j); the V producer refills the stage only after PV(j),
+        // i.e. after this tile's P, so one phase is pending
+        const int sst = j % NCS_V;
+        if (!(ok = mbar_wait_warp(&sc_full[sst], (j / NCS_V) & 1, SITE_DC_SM_V))) break;
+        const float ks = scales[sst * 256 + t], vs = scales[sst * 256 + 128 + t];
         if (!(ok = mbar_wait_warp(&s_full[bs], (j / NS) & 1, SITE_DC_SM_S))) break;
         if (t == 0) ATTN_EVT(j, 4);
         tc_fence_after();

@@ -157,6 +157,12 @@ __device__ __forceinline__ void cp_async_16_zfill(void* dst, const void* src, ui
                : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared that reads src_bytes (0 or 4) and zero-fills the rest.
+__device__ __forceinline__ void cp_async_4_zfill(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
 // The barrier tracks this thread's earlier cp.async copies: its pending count goes up by one now
 // and comes back down by an arrival once those copies have landed (net zero arrivals).
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {

@@ -9,6 +9,7 @@ namespace attn {
 enum DeviceErrorCode : uint32_t {
   ATTN_DEV_OK = 0,
   ATTN_DEV_TIMEOUT = 1,  // a bounded wait ran out
+  ATTN_DEV_BAD_PAGE = 2,  // a decode page-table entry outside [0, num_pages)
 };
 
 // Wait sites, recorded with the error so a timeout names the wait that gave up.
@@ -36,6 +37,7 @@ enum WaitSite : int {
   SITE_DC_MMA_O = 41,
   SITE_DC_MMA_S = 42,
   SITE_DC_SM_P = 43,
+  SITE_DC_PAGE = 44,
 };
 
 // (code << 16) | site of the first error since the last reset; 0 when clean.

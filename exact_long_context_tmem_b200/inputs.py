@@ -162,6 +162,45 @@ def decode_inputs(w: Workload, B: int | None = None, Tmax: int | None = None, se
     return out
 
 
+def paged_inputs(d: dict, page_size: int, seed: int, spare_frac: float = 0.125):
+    """Lay a decode_inputs() cache out as a page pool plus a page table (no arithmetic, only
+    copies).  Each sequence's pages covering [0, len) go to pool pages in a seeded random order;
+    table entries past them are -1; a few spare pool pages and every slot past a length hold
+    the padding (NaN, code 0x7f for FP8), so any read of an unmapped page shows up.
+
+    Returns a dict with q, kv_lens, page_table int32 [B, max_pages], page_size, num_pages and
+    k_pool, v_pool [num_pages, page_size, Hkv, D] (bf16) or k_codes/v_codes pools with
+    k_scale/v_scale pools [num_pages, page_size, Hkv].
+    """
+    fp8 = "k_codes" in d
+    names = ("k_codes", "v_codes", "k_scale", "v_scale") if fp8 else ("k", "v")
+    lens = d["kv_lens"].long()
+    B, Tmax = d[names[0]].shape[0], d[names[0]].shape[1]
+    max_pages = (Tmax + page_size - 1) // page_size
+    need = [(int(x) + page_size - 1) // page_size for x in lens]
+    total = sum(need)
+    spare = max(2, int(total * spare_frac))
+    g = generator(seed)
+    perm = torch.randperm(total + spare, generator=g)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    out = {"q": d["q"], "kv_lens": d["kv_lens"], "page_size": page_size, "num_pages": total + spare}
+    for name in names:
+        src = d[name]
+        pad_val = 0x7F if src.dtype == torch.uint8 else float("nan")
+        pool = torch.full((total + spare, page_size) + tuple(src.shape[2:]), pad_val, dtype=src.dtype)
+        padded = torch.full((B, max_pages * page_size) + tuple(src.shape[2:]), pad_val, dtype=src.dtype)
+        padded[:, :Tmax] = src
+        k = 0
+        for b in range(B):
+            for i in range(need[b]):
+                pool[perm[k]] = padded[b, i * page_size:(i + 1) * page_size]
+                table[b, i] = int(perm[k])
+                k += 1
+        out[name] = pool
+    out["page_table"] = table
+    return out
+
+
 def sample_rows(S: int, n_random: int, seed: int, edges=()) -> list[int]:
     """Seeded query-row sample for checks on workloads too big for the full oracle."""
     g = generator(seed)

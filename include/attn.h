@@ -119,6 +119,33 @@ ATTN_API attn_status_t attn_decode_splitkv(const void* q, const void* k, const v
                                   size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * attn_decode_paged — attn_decode_splitkv over a paged KV cache.
+ *
+ * [COOPT] Opt-Pa: sequences are cut into fixed-size pages (e.g. 512 tokens) and only pages that
+ * are mapped are ever touched ("lazy mapping").  Here the cache is a pool of pages shared by all
+ * sequences and a page table maps sequence b's logical page i (tokens i*page_size .. +page_size-1)
+ * to a pool page.  Only the pages covering [0, kv_lens[b]) are read; table entries past them are
+ * never read and may hold anything (-1 for unmapped).  Same split-KV method, outputs, scaling and
+ * workspace rule as attn_decode_splitkv, with Tmax = max_pages * page_size.
+ *
+ *   q                 device bf16 [B, Hq, D]
+ *   k_pool, v_pool    device [num_pages, page_size, Hkv, D]: bf16 or E4M3 codes (kv_dtype)
+ *   k_scale_pool, v_scale_pool  device float32 [num_pages, page_size, Hkv] for FP8, else NULL
+ *   page_table        device int32 [B, max_pages]; entries used must lie in [0, num_pages)
+ *   page_size         a multiple of 128 (a 128-token tile never straddles two pages)
+ *   kv_lens           device int32 [B], each in [0, max_pages * page_size]
+ *   num_splits, o, lse, ws, ws_bytes, stream  as for attn_decode_splitkv; the workspace size is
+ *                     attn_decode_workspace_bytes(dims, max_pages * page_size, num_splits)
+ * Errors: ATTN_ERR_INVALID_ARG for bad sizes, null or misaligned pointers; a page-table entry
+ * outside [0, num_pages) met on the device is never dereferenced (its tokens read as zeros) and
+ * is reported later by attn_device_status as ATTN_ERR_INVALID_ARG (site 44).
+ * ------------------------------------------------------------------------------------------ */
+ATTN_API attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, attn_dtype_t kv_dtype,
+                                const float* k_scale_pool, const float* v_scale_pool, const int* page_table,
+                                int max_pages, int page_size, int num_pages, const int* kv_lens, attn_dims_t dims,
+                                int num_splits, void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * attn_decode_splitkv_noalloc — the same split-KV decode, for callers that cannot allocate.
  *
  * The pages have no counterpart to this entry point; it is an integration aid.  Some callers
@@ -214,8 +241,9 @@ ATTN_API const char* attn_status_string(attn_status_t status);
 /* Last CUDA error code seen by this host thread inside the library (0 = none). */
 ATTN_API int attn_last_cuda_error(void);
 /* Reads the device status word of the current device (synchronises the device).  Returns
- * ATTN_ERR_TIMEOUT if a kernel's bounded wait ran out since the last reset, and stores the
- * wait site in *site when site != NULL.  reset != 0 clears the word. */
+ * ATTN_ERR_TIMEOUT if a kernel's bounded wait ran out since the last reset, ATTN_ERR_INVALID_ARG
+ * if a decode kernel met a page-table entry outside the pool, and stores the site in *site when
+ * site != NULL.  reset != 0 clears the word. */
 ATTN_API attn_status_t attn_device_status(int reset, int* site);
 /* Upper bound of any single in-kernel wait, in nanoseconds (default 2e9). */
 ATTN_API attn_status_t attn_set_wait_limit_ns(unsigned long long ns);

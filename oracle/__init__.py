@@ -9,4 +9,5 @@ Modules:
   attention  exact attention rows, single-token decode, log-sum-exp merge
   fp8        E4M3 code table from the format definition
   stream     exact-cover check of a (query block, key chunk) task list
+  paged      paged KV cache: gather mapped pages into the contiguous cache, then decode
 """

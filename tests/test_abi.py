@@ -97,6 +97,22 @@ def test_decode_unsupported(L):
     assert L.attn_decode_splitkv(*args, _dims(Hq=34, Hkv=2, D=128), 1, FAKE, None, None, 0, None) == 2
 
 
+@pytest.mark.parametrize("case", [
+    dict(page_size=100), dict(page_size=64), dict(max_pages=0), dict(num_pages=0), dict(page_table=None),
+    dict(k_pool=None), dict(q=None), dict(kv_lens=None), dict(kv_dtype=7), dict(k_scale=FAKE),
+    dict(kv_dtype=1), dict(ws=None), dict(num_splits=-1), dict(page_table=ctypes.c_void_p(0x10002)),
+])
+def test_decode_paged_invalid_args(L, case):
+    a = dict(q=FAKE, k_pool=FAKE, v_pool=FAKE, kv_dtype=0, k_scale=None, v_scale=None, page_table=FAKE,
+             max_pages=8, page_size=512, num_pages=64, kv_lens=FAKE, dims=_dims(D=128), num_splits=4, o=FAKE,
+             lse=None, ws=FAKE, ws_bytes=1 << 30)
+    a.update(case)
+    st = L.attn_decode_paged(a["q"], a["k_pool"], a["v_pool"], a["kv_dtype"], a["k_scale"], a["v_scale"],
+                             a["page_table"], a["max_pages"], a["page_size"], a["num_pages"], a["kv_lens"],
+                             a["dims"], a["num_splits"], a["o"], a["lse"], a["ws"], a["ws_bytes"], None)
+    assert st == 1
+
+
 def test_decode_workspace_and_splits(L):
     d = _dims(B=4, Hq=32, Hkv=8, D=128)
     for P in (1, 2, 7, 19):
