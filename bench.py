@@ -287,9 +287,10 @@ def bench_prefill(w, steps, warmup, world, dev, pk):
 PAGE_SIZE = 512
 
 
-def bench_decode(name, steps, warmup, world, dev, pk, paged=False):
+def bench_decode(name, steps, warmup, world, dev, pk, paged=False, n_q=1):
     """Split-KV decode of a decode workload; paged=True lays the same cache out as a pool of
-    PAGE_SIZE-token pages in seeded random order with a page table (attn_decode_paged)."""
+    PAGE_SIZE-token pages in seeded random order with a page table (attn_decode_paged); n_q > 1
+    decodes the last n_q cache tokens of every sequence in one pass (attn_decode_multi)."""
     from exact_long_context_tmem_b200 import attn as A
 
     w = I.WORKLOADS[name]
@@ -307,14 +308,18 @@ def bench_decode(name, steps, warmup, world, dev, pk, paged=False):
     else:
         kd, vd = d["k"].to(dev), d["v"].to(dev)
         ks = vs = None
-    o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
-    nbytes = A.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, Tmax)
+    if n_q > 1:
+        qd = I.randn_bf16((w.B, n_q, w.Hq, w.D), I.generator(w.seed + 11)).to(dev)
+    o = torch.empty((w.B, n_q, w.Hq, w.D) if n_q > 1 else (w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, n_q, w.Hq) if n_q > 1 else (w.B, w.Hq), dtype=torch.float32, device=dev)
+    nbytes = A.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, Tmax) * n_q
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
     splits = A.attn_decode_num_splits(w.B, w.Hq, w.Hkv, w.D, Tmax)
 
     def step():
-        if paged:
+        if n_q > 1:
+            A.attn_decode_multi(qd, kd, vd, ld, k_scale=ks, v_scale=vs, o=o, lse=lse, ws=ws)
+        elif paged:
             A.attn_decode_paged(qd, kd, vd, table, ld, k_scale=ks, v_scale=vs, o=o, lse=lse, ws=ws)
         else:
             A.attn_decode_splitkv(qd, kd, vd, ld, k_scale=ks, v_scale=vs, o=o, lse=lse, ws=ws)
@@ -333,11 +338,13 @@ def bench_decode(name, steps, warmup, world, dev, pk, paged=False):
     call_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
     nb = decode_bytes(w, lens)
     gbs = nb / (call_ms * 1e-3) / 1e9
-    return {"workload": name + (f"_paged{PAGE_SIZE}" if paged else ""), "value": round(gbs * world, 1), "unit": "GB/s",
+    suffix = (f"_paged{PAGE_SIZE}" if paged else "") + (f"_multi{n_q}" if n_q > 1 else "")
+    return {"workload": name + suffix, "value": round(gbs * world, 1), "unit": "GB/s",
             "ms_per_step": round(call_ms, 4),
             "splits": splits, "kv_tokens": int(lens.sum()), "bytes_per_step": nb,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": None if paged else ncu_traffic(name),
+                         "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "traffic": None if (paged or n_q > 1) else ncu_traffic(name),
                          "timed": "split kernel + merge kernel (one API call)"},
             "launches": steps * (2 if splits > 1 else 1)}
 
@@ -401,7 +408,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--stream", action="store_true", help="also run the 1M-token streamed prefill")
     ap.add_argument("--cpu-rows", type=int, default=128)
-    ap.add_argument("--workloads", default="prefill,decode_bf16,decode_fp8,decode_bf16_paged,decode_fp8_paged",
+    ap.add_argument("--workloads",
+                    default="prefill,decode_bf16,decode_fp8,decode_bf16_paged,decode_fp8_paged,decode_bf16_multi,decode_fp8_multi",
                     help="comma list of prefill, decode_bf16, decode_fp8 (profiling runs select one)")
     args = ap.parse_args()
     w = I.WORKLOADS[HEADLINE]
@@ -450,6 +458,8 @@ def main():
                 dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk))
             if key + "_paged" in sel:
                 dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk, paged=True))
+            if key + "_multi" in sel:
+                dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk, n_q=4))
     st, site = A.attn_device_status(reset=True)
     if st != 0:
         raise SystemExit(f"device status {st} at wait site {site}")

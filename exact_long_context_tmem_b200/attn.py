@@ -25,7 +25,7 @@ ATTN_BF16, ATTN_FP8_E4M3, ATTN_F32 = 0, 1, 2
 
 EXPORTS = [
     "attn_prefill", "attn_decode_workspace_bytes", "attn_decode_num_splits", "attn_decode_splitkv",
-    "attn_decode_splitkv_noalloc", "attn_decode_paged",
+    "attn_decode_splitkv_noalloc", "attn_decode_paged", "attn_decode_multi", "attn_decode_multi_workspace_bytes",
     "attn_merge_lse", "attn_stream_plan", "attn_stream_task", "attn_chunked_stream", "attn_status_string",
     "attn_last_cuda_error", "attn_device_status", "attn_set_wait_limit_ns", "attn_debug_wait_probe",
     "attn_debug_inject", "attn_debug_exp2",
@@ -77,6 +77,10 @@ def lib() -> ctypes.CDLL:
     L.attn_decode_splitkv_noalloc.restype = i
     L.attn_decode_paged.argtypes = [vp, vp, vp, i, vp, vp, vp, i, i, i, vp, Dims, i, vp, vp, vp, sz, vp]
     L.attn_decode_paged.restype = i
+    L.attn_decode_multi_workspace_bytes.argtypes = [Dims, i, i, i]
+    L.attn_decode_multi_workspace_bytes.restype = sz
+    L.attn_decode_multi.argtypes = [vp, vp, vp, i, vp, vp, vp, i, i, Dims, i, vp, vp, vp, sz, vp]
+    L.attn_decode_multi.restype = i
     L.attn_merge_lse.argtypes = [vp, vp, i, ll, i, vp, i, vp, i, vp]
     L.attn_merge_lse.restype = i
     L.attn_stream_plan.argtypes = [Dims, ll, i, ll, sz, ctypes.POINTER(StreamPlan)]
@@ -179,6 +183,31 @@ def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: 
                                    _ptr(v_scale), _ptr(kv_lens), int(Tmax), dims, int(num_splits), _ptr(o),
                                    _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_decode_multi(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: float | None = None,
+                      num_splits: int = 0, o=None, lse=None, ws=None, want_lse: bool = True, stream=None):
+    """q [B,n_q,Hq,D] bf16 (n_q new tokens per sequence, already in the cache); k/v as for
+    attn_decode_splitkv -> (o [B,n_q,Hq,D] bf16, lse [B,n_q,Hq] float32)."""
+    _need_cuda(q, k, v, kv_lens, k_scale, v_scale)
+    B, n_q, Hq, D = q.shape
+    Tmax, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    fp8 = k.dtype in (torch.uint8, torch.float8_e4m3fn)
+    dims = _dims(B, Hq, Hkv, D, scale)
+    if o is None:
+        o = torch.empty((B, n_q, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q, Hq), dtype=torch.float32, device=q.device)
+    need = int(lib().attn_decode_multi_workspace_bytes(dims, int(Tmax), int(n_q), int(num_splits)))
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().attn_decode_multi(_ptr(q), _ptr(k), _ptr(v), ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(k_scale),
+                                 _ptr(v_scale), _ptr(kv_lens), int(Tmax), int(n_q), dims, int(num_splits), _ptr(o),
+                                 _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
+    _check(st, "attn_decode_multi")
     return o, lse
 
 

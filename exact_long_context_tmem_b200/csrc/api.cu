@@ -175,9 +175,9 @@ static int decode_split_tokens(int Tmax, int P) {
   return ((Tmax + P - 1) / P + 127) / 128 * 128;
 }
 
-static size_t decode_ws_bytes(const attn_dims_t& d, int P) {
+static size_t decode_ws_bytes(const attn_dims_t& d, int P, int n_q = 1) {
   if (P <= 1) return 0;
-  const size_t rows = (size_t)P * d.B * d.Hq;
+  const size_t rows = (size_t)P * d.B * n_q * d.Hq;
   return rows * d.D * sizeof(float) + rows * sizeof(float) + 256;
 }
 
@@ -213,7 +213,8 @@ struct DecodePaging {
 template <bool FP8>
 static attn_status_t launch_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
                                    const int* kv_lens, int Tmax, const attn_dims_t& d, int P, int split_tokens,
-                                   void* o, float* lse, void* ws, cudaStream_t stream, const DecodePaging& pg) {
+                                   void* o, float* lse, void* ws, cudaStream_t stream, const DecodePaging& pg,
+                                   int n_q = 1) {
   attn_status_t st;
   CUtensorMap mk, mv;
   // With Tmax == 0 every split is empty and no map is read; it still needs a valid base and extent.
@@ -234,6 +235,7 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   p.Hq = d.Hq;
   p.Hkv = d.Hkv;
   p.G = d.Hq / d.Hkv;
+  p.n_q = n_q;
   p.Tmax = Tmax;
   p.split_tokens = split_tokens;
   p.n_splits = P;
@@ -248,7 +250,7 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   p.page_size = std::max(pg.page_size, 1);
   p.num_pages = pg.num_pages;
   float* ws_f = reinterpret_cast<float*>(ws);
-  const size_t rows = (size_t)P * d.B * d.Hq;
+  const size_t rows = (size_t)P * d.B * n_q * d.Hq;
   p.o_part = P > 1 ? ws_f : nullptr;
   p.lse_part = P > 1 ? ws_f + rows * 128 : nullptr;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
@@ -256,10 +258,11 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   dim3 grid(P, d.Hkv, d.B);
   if ((long long)P * d.Hkv * d.B > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;  // work items are int-indexed
   // The query group is padded to the next power of two (<= 16) so the kernels' per-row loops unroll.
-  if (p.G <= 1) st = launch_decode_gp<FP8, 1>(mk, mv, p, grid, stream);
-  else if (p.G <= 2) st = launch_decode_gp<FP8, 2>(mk, mv, p, grid, stream);
-  else if (p.G <= 4) st = launch_decode_gp<FP8, 4>(mk, mv, p, grid, stream);
-  else if (p.G <= 8) st = launch_decode_gp<FP8, 8>(mk, mv, p, grid, stream);
+  const int R = p.G * n_q;  // MMA rows of one (sequence, KV head)
+  if (R <= 1) st = launch_decode_gp<FP8, 1>(mk, mv, p, grid, stream);
+  else if (R <= 2) st = launch_decode_gp<FP8, 2>(mk, mv, p, grid, stream);
+  else if (R <= 4) st = launch_decode_gp<FP8, 4>(mk, mv, p, grid, stream);
+  else if (R <= 8) st = launch_decode_gp<FP8, 8>(mk, mv, p, grid, stream);
   else st = launch_decode_gp<FP8, 16>(mk, mv, p, grid, stream);
   if (st != ATTN_OK) return st;
   if (P > 1) {
@@ -267,7 +270,7 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
     mp.o_parts = p.o_part;
     mp.lse_parts = p.lse_part;
     mp.P = P;
-    mp.R = (long long)d.B * d.Hq;
+    mp.R = (long long)d.B * n_q * d.Hq;
     mp.o_out = o;
     mp.o_f32 = 0;
     mp.lse_out = lse;
@@ -426,6 +429,36 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v
     return launch_decode<true>(q, k_pool, v_pool, k_scale_pool, v_scale_pool, kv_lens, Tmax, dims, P, per, o, lse, ws,
                                st, pg);
   return launch_decode<false>(q, k_pool, v_pool, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
+}
+
+size_t attn_decode_multi_workspace_bytes(attn_dims_t dims, int Tmax, int n_q, int num_splits) {
+  if (!dims_ok(dims) || Tmax < 0 || n_q < 1) return 0;
+  return decode_ws_bytes(dims, decode_splits(dims, Tmax, num_splits), n_q);
+}
+
+attn_status_t attn_decode_multi(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax, int n_q,
+                                attn_dims_t dims, int num_splits, void* o, float* lse, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (!dims_ok(dims) || Tmax < 0 || num_splits < 0 || num_splits > 4096 || n_q < 1) return ATTN_ERR_INVALID_ARG;
+  if (kv_dtype != ATTN_BF16 && kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (dims.B == 0) return ATTN_OK;
+  if (!q || !o || !kv_lens || (Tmax > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  const bool fp8 = kv_dtype == ATTN_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr) || fp8 != (v_scale != nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned4(kv_lens) || (lse && !aligned4(lse))) return ATTN_ERR_INVALID_ARG;
+  if (Tmax > 0 && (!aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
+  if (fp8 && (!aligned4(k_scale) || !aligned4(v_scale))) return ATTN_ERR_INVALID_ARG;
+  if (dims.D != 128 || (long long)(dims.Hq / dims.Hkv) * n_q > 16) return ATTN_ERR_UNSUPPORTED;
+  if (dims.B > 65535 || dims.Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  const int P = decode_splits(dims, Tmax, num_splits);
+  const size_t need = decode_ws_bytes(dims, P, n_q);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int per = decode_split_tokens(Tmax, P);
+  const DecodePaging pg{nullptr, 1, Tmax, dims.B};
+  if (fp8) return launch_decode<true>(q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg, n_q);
+  return launch_decode<false>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg, n_q);
 }
 
 // Split-KV decode without allocation: the split partials live in this static device array

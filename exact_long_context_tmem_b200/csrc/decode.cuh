@@ -28,10 +28,15 @@ namespace attn {
 
 struct DecodeParams {
   int B, Hq, Hkv, G, Tmax;
+  // Query tokens per sequence (1 for plain decode).  With n_q > 1 (multi-token decode / draft
+  // verification, ORT GQA analysis "Verification"), token i of sequence b sits at position
+  // len_b - n_q + i and sees keys [0, len_b - n_q + i + 1); its G heads are MMA rows
+  // r = i * G + g, so the rows of one (sequence, KV head) are n_q * G <= 16.
+  int n_q;
   int split_tokens;  // tokens per split, multiple of 128
   int n_splits;
   float scale_log2;
-  const __nv_bfloat16* q;  // [B, Hq, 128]
+  const __nv_bfloat16* q;  // [B, n_q, Hq, 128]
   const float* k_scale;    // [B, Tmax, Hkv] (FP8) or null
   const float* v_scale;
   const int* kv_lens;       // [B]
@@ -41,11 +46,26 @@ struct DecodeParams {
   // is one page of Tmax tokens per sequence (page_size = Tmax, num_pages = B, page of b = b).
   const int* page_table;    // device int32 [B, max_pages] or null
   int max_pages, page_size, num_pages;
-  float* o_part;            // [n_splits, B, Hq, 128] when n_splits > 1
-  float* lse_part;          // [n_splits, B, Hq]
-  __nv_bfloat16* o;         // [B, Hq, 128] when n_splits == 1
-  float* lse;               // [B, Hq] or null
+  float* o_part;            // [n_splits, B * n_q * Hq, 128] when n_splits > 1
+  float* lse_part;          // [n_splits, B * n_q * Hq]
+  __nv_bfloat16* o;         // [B, n_q, Hq, 128] when n_splits == 1
+  float* lse;               // [B, n_q, Hq] or null
 };
+
+// Rows of one (sequence, KV head): n_q query tokens x G heads.
+__device__ __forceinline__ int decode_rows(const DecodeParams& p) { return p.n_q * p.G; }
+
+// Row r = i * G + g of (sequence b, KV head kvh) in the [B, n_q, Hq] order of q, o and lse.
+__device__ __forceinline__ long long decode_row_index(const DecodeParams& p, int b, int kvh, int r) {
+  const int i = r / p.G, g = r - i * p.G;
+  return ((long long)b * p.n_q + i) * p.Hq + (long long)kvh * p.G + g;
+}
+
+// Exclusive key limit of row r within a split ending at t1: the token's causal limit, and t1.
+__device__ __forceinline__ int decode_row_limit(const DecodeParams& p, int len, int t1, int r) {
+  const int lim = len - p.n_q + 1 + r / p.G;
+  return lim < t1 ? lim : t1;
+}
 
 // Pool page of the tile of sequence b that starts at token tok (a multiple of 128; with a table,
 // page_size is a multiple of 128, so a tile never straddles two pages).  Table entries are read
@@ -181,7 +201,8 @@ __device__ __forceinline__ bool decode_softmax_core(DecodeRows<GP>& rows, const 
 // bf16 decode: the 16 S^T columns of this lane, scaled by sc (log2 domain), then the shared core.
 template <int GP, bool F16P>
 __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j, bool has_prev, int lane, int wq,
-                                                    int t, bool valid, float sc, float vs, uint32_t tS_lane,
+                                                    int t, int tok, const int (&rlim)[GP], float sc, float vs,
+                                                    uint32_t tS_lane,
                                                     uint32_t tO_lane, float* red_max, uint64_t* red_bar,
                                                     uint64_t* prev_pv, uint32_t prev_pv_parity, uint8_t* p_tile,
                                                     float threshold) {
@@ -190,7 +211,7 @@ __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j,
   tmem_wait_ld();
   float x[GP];
 #pragma unroll
-  for (int g = 0; g < GP; ++g) x[g] = valid ? __uint_as_float(sv[g]) * sc : -INFINITY;
+  for (int g = 0; g < GP; ++g) x[g] = tok < rlim[g] ? __uint_as_float(sv[g]) * sc : -INFINITY;
   return decode_softmax_core<GP, F16P>(rows, x, j, has_prev, lane, wq, t, vs, tO_lane, red_max, red_bar, prev_pv,
                                        prev_pv_parity, p_tile, threshold);
 }
@@ -224,27 +245,29 @@ __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const Deco
     mbar_arrive(o_free);
   }
   float my_lse = -INFINITY;
+  const int R = decode_rows(p);
+  const long long rows_all = (long long)p.B * p.n_q * p.Hq;
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
-    if (g < G) {
+    if (g < R) {
       const float l = red_sum[g] + red_sum[16 + g] + red_sum[32 + g] + red_sum[48 + g];
       const float ov = (l > 0.f) ? __uint_as_float(orow[g]) / l : 0.f;
       const float lse = (l > 0.f) ? (rows.m_used[g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (g == t) my_lse = lse;
-      const long long h = (long long)kvh * G + g;
+      const long long h = decode_row_index(p, b, kvh, g);
       if (p.n_splits == 1) {
-        p.o[((long long)b * p.Hq + h) * D + t] = __float2bfloat16_rn(ov);
+        p.o[h * D + t] = __float2bfloat16_rn(ov);
       } else {
-        p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + t] = ov;
+        p.o_part[((long long)split * rows_all + h) * D + t] = ov;
       }
     }
   }
-  if (t < G) {
-    const long long h = (long long)kvh * G + t;
+  if (t < R) {
+    const long long h = decode_row_index(p, b, kvh, t);
     if (p.n_splits == 1) {
-      if (p.lse) p.lse[(long long)b * p.Hq + h] = my_lse;
+      if (p.lse) p.lse[h] = my_lse;
     } else {
-      p.lse_part[((long long)split * p.B + b) * p.Hq + h] = my_lse;
+      p.lse_part[(long long)split * rows_all + h] = my_lse;
     }
   }
   return true;
@@ -254,25 +277,27 @@ __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const Deco
 __device__ __forceinline__ void decode_write_empty(const DecodeParams& p, int G, int split, int kvh, int b, int tid,
                                                    int nthreads) {
   constexpr int D = 128;
-  for (int i = tid; i < G * D; i += nthreads) {
+  const long long rows_all = (long long)p.B * p.n_q * p.Hq;
+  for (int i = tid; i < decode_rows(p) * D; i += nthreads) {
     const int g = i / D, d = i % D;
-    const long long h = (long long)kvh * G + g;
+    const long long h = decode_row_index(p, b, kvh, g);
     if (p.n_splits == 1) {
-      p.o[((long long)b * p.Hq + h) * D + d] = __float2bfloat16_rn(0.f);
-      if (d == 0 && p.lse) p.lse[(long long)b * p.Hq + h] = -INFINITY;
+      p.o[h * D + d] = __float2bfloat16_rn(0.f);
+      if (d == 0 && p.lse) p.lse[h] = -INFINITY;
     } else {
-      p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + d] = 0.f;
-      if (d == 0) p.lse_part[((long long)split * p.B + b) * p.Hq + h] = -INFINITY;
+      p.o_part[((long long)split * rows_all + h) * D + d] = 0.f;
+      if (d == 0) p.lse_part[(long long)split * rows_all + h] = -INFINITY;
     }
   }
 }
 
-// Chunk c (< 256) of the query group: row g = c / 16, elements 8 (c % 16) .. + 7 (zero for g >= G).
+// Chunk c (< 256) of the query rows: row r = c / 16, elements 8 (c % 16) .. + 7 (zero for r past
+// the n_q * G rows).
 __device__ __forceinline__ uint4 decode_q_chunk_load(const DecodeParams& p, int G, int kvh, int b, int c) {
   constexpr int D = 128;
-  const int g = c >> 4, cc = c & 15;
+  const int r = c >> 4, cc = c & 15;
   uint4 x = make_uint4(0u, 0u, 0u, 0u);
-  if (g < G) x = *reinterpret_cast<const uint4*>(p.q + ((long long)b * p.Hq + (long long)kvh * G + g) * D + cc * 8);
+  if (r < p.n_q * G) x = *reinterpret_cast<const uint4*>(p.q + decode_row_index(p, b, kvh, r) * D + cc * 8);
   return x;
 }
 
@@ -478,22 +503,25 @@ __global__ void __launch_bounds__(192, 1)
     mbar_arrive(q_ready);
 
     DecodeRows<GP> rows;
+    int rlim[GP];  // per-row exclusive key limits (a query token sees its own causal prefix)
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       rows.m_used[g] = -INFINITY;
       rows.l_part[g] = 0.f;
+      rlim[g] = g < decode_rows(p) ? decode_row_limit(p, len, t1, g) : t1;
     }
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
       const int st = j % C::NST;
       const uint32_t ph = (j / C::NST) & 1;
-      const bool valid = t0 + j * 128 + t < t1;
+      const int tok = t0 + j * 128 + t;
+      const bool valid = tok < t1;
       // tcgen05.ld/st are warp-collective: every lane takes the same branch around them.
       if (!(ok = mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, SITE_DC_SM_S))) break;
       tc_fence_after();
       // PV(j-1) is the j-th completion of o_ready; S(j) completing implies PV(j-2) done, so at
       // most one phase is pending and the parity wait is unambiguous.
-      if (!(ok = decode_softmax_tile<GP, false>(rows, j, j > 0, lane, wq, t, valid, p.scale_log2, 1.f,
+      if (!(ok = decode_softmax_tile<GP, false>(rows, j, j > 0, lane, wq, t, tok, rlim, p.scale_log2, 1.f,
                                                 tS0 + (j & 1) * 16 + lane_off, tO + lane_off, red_max, red_bar,
                                                 o_ready, (j - 1) & 1, smem + C::OFF_P + (j & 1) * C::P_BYTES,
                                                 C::RESCALE_THRESHOLD)))

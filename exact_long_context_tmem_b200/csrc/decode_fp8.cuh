@@ -87,6 +87,7 @@ struct DecodeFp8Cfg {
 // One work item of the persistent decode: a split of one (sequence, KV head).
 struct DecodeItem {
   int split, kvh, b;
+  int len;     // the sequence's length
   int t0, t1;  // token range [t0, t1)
   int n;       // 128-token tiles (0: empty split)
 };
@@ -98,6 +99,7 @@ __device__ __forceinline__ DecodeItem decode_item(const DecodeParams& p, int w) 
   it.b = w / (p.n_splits * p.Hkv);
   int len = __ldg(p.kv_lens + it.b);
   len = len < 0 ? 0 : (len > p.Tmax ? p.Tmax : len);
+  it.len = len;
   it.t0 = it.split * p.split_tokens;
   it.t1 = min(len, it.t0 + p.split_tokens);
   it.n = it.t1 > it.t0 ? (it.t1 - it.t0 + 127) / 128 : 0;
@@ -239,7 +241,8 @@ __device__ __forceinline__ uint32_t p8_offset(int r, int t) {
 // that completes with the previous PV.  Returns false, warp-uniformly, if a bounded wait ran out.
 template <int GP, int NQ, int NP, int NS>
 __device__ __forceinline__ bool fp8_softmax_tile(DecodeRows<GP>& rows, int j, bool has_prev, int lane, int wq, int t,
-                                                 bool valid, float sck, float vs, const float (&fq)[GP],
+                                                 int tok, const int (&rlim)[GP], float sck, float vs,
+                                                 const float (&fq)[GP],
                                                  uint32_t tS_lane, uint32_t tO_lane, float* red_max,
                                                  uint64_t* red_bar, uint64_t* s_free, uint64_t* pv_done,
                                                  uint8_t* p_tile, float threshold) {
@@ -253,7 +256,7 @@ __device__ __forceinline__ bool fp8_softmax_tile(DecodeRows<GP>& rows, int j, bo
   for (int g = 0; g < GP; ++g) {
     const float s12 = fmaf(__uint_as_float(sv[2 * GP + g]), 0.0625f, __uint_as_float(sv[GP + g]));
     const float s = fmaf(s12, 0.0625f, __uint_as_float(sv[g]));
-    x[g] = valid ? s * (sck * fq[g]) : -INFINITY;
+    x[g] = tok < rlim[g] ? s * (sck * fq[g]) : -INFINITY;
     y[g] = x[g] + lv;
   }
   float* rm = red_max + (j & 1) * 64;
@@ -338,9 +341,11 @@ __device__ __forceinline__ bool fp8_epilogue(DecodeRows<GP>& rows, const DecodeP
   tc_fence_before();
   mbar_arrive(o_free);
   float my_lse = -INFINITY;
+  const int R = decode_rows(p);
+  const long long rows_all = (long long)p.B * p.n_q * p.Hq;
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
-    if (g < G) {
+    if (g < R) {
       const float l = red_sum[g] + red_sum[16 + g] + red_sum[32 + g] + red_sum[48 + g];
       const float c23 = fmaf(__uint_as_float(o[3 * GP + g]), 0.0625f, __uint_as_float(o[2 * GP + g]));
       const float c123 = fmaf(c23, 0.0625f, __uint_as_float(o[GP + g]));
@@ -348,20 +353,20 @@ __device__ __forceinline__ bool fp8_epilogue(DecodeRows<GP>& rows, const DecodeP
       const float ov = (l > 0.f) ? acc / l : 0.f;
       const float lse = (l > 0.f) ? (rows.m_used[g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (g == t) my_lse = lse;
-      const long long h = (long long)kvh * G + g;
+      const long long h = decode_row_index(p, b, kvh, g);
       if (p.n_splits == 1) {
-        p.o[((long long)b * p.Hq + h) * D + t] = __float2bfloat16_rn(ov);
+        p.o[h * D + t] = __float2bfloat16_rn(ov);
       } else {
-        p.o_part[(((long long)split * p.B + b) * p.Hq + h) * D + t] = ov;
+        p.o_part[((long long)split * rows_all + h) * D + t] = ov;
       }
     }
   }
-  if (t < G) {
-    const long long h = (long long)kvh * G + t;
+  if (t < R) {
+    const long long h = decode_row_index(p, b, kvh, t);
     if (p.n_splits == 1) {
-      if (p.lse) p.lse[(long long)b * p.Hq + h] = my_lse;
+      if (p.lse) p.lse[h] = my_lse;
     } else {
-      p.lse_part[((long long)split * p.B + b) * p.Hq + h] = my_lse;
+      p.lse_part[(long long)split * rows_all + h] = my_lse;
     }
   }
   return true;
@@ -715,9 +720,12 @@ __global__ void __launch_bounds__(256, 1)
         rows.l_part[g] = 0.f;
       }
       const uint32_t tO = tO0 + (ie & 1) * NP + lane_off;
+      int rlim[GP];  // per-row exclusive key limits (a query token sees its own causal prefix)
+#pragma unroll
+      for (int g = 0; g < GP; ++g) rlim[g] = g < decode_rows(p) ? decode_row_limit(p, cur.len, cur.t1, g) : cur.t1;
       for (int l = 0; l < cur.n; ++l, ++j) {
         const int bs = j % NS;
-        const bool valid = cur.t0 + l * 128 + t < cur.t1;
+        const int tok = cur.t0 + l * 128 + t;
         // scales of tile j: staged with V(j); the V producer refills the stage only after PV(j),
         // i.e. after this tile's P, so one phase is pending
         const int sst = j % NCS_V;
@@ -726,7 +734,7 @@ __global__ void __launch_bounds__(256, 1)
         if (!(ok = mbar_wait_warp(&s_full[bs], (j / NS) & 1, SITE_DC_SM_S))) break;
         if (t == 0) ATTN_EVT(j, 4);
         tc_fence_after();
-        if (!(ok = fp8_softmax_tile<GP, NQ, NP, NS>(rows, j, l > 0, lane, wq, t, valid, p.scale_log2 * ks, vs, fq,
+        if (!(ok = fp8_softmax_tile<GP, NQ, NP, NS>(rows, j, l > 0, lane, wq, t, tok, rlim, p.scale_log2 * ks, vs, fq,
                                                     tS0 + bs * NQ + lane_off, tO, red_max, red_bar, s_free, pv_done,
                                                     smem + C::OFF_P + bs * C::P_BYTES, C::RESCALE_THRESHOLD)))
           break;

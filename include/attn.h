@@ -119,6 +119,27 @@ ATTN_API attn_status_t attn_decode_splitkv(const void* q, const void* k, const v
                                   size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * attn_decode_multi — n_q query tokens per sequence over one KV cache (multi-token decode,
+ * e.g. verifying n_q draft tokens).
+ *
+ * [ORT-GQA] Code analysis 4 (packed QKV with past lengths): a new token's absolute position is
+ * the past length plus its index among the new tokens.  Here the cache already holds the n_q
+ * new tokens, so token i of sequence b sits at position kv_lens[b] - n_q + i and sees keys
+ * [0, kv_lens[b] - n_q + i + 1) (a token with no visible key gets O = 0, LSE = -inf).  One pass
+ * over the cache serves all n_q tokens: their n_q * Hq/Hkv query rows share each K/V tile, which
+ * requires n_q * Hq/Hkv <= 16.  n_q = 1 is attn_decode_splitkv.
+ *
+ *   q      device bf16 [B, n_q, Hq, D];  o device bf16 [B, n_q, Hq, D];  lse float32 [B, n_q, Hq]
+ *   ws     at least attn_decode_multi_workspace_bytes(dims, Tmax, n_q, num_splits) bytes
+ *   other arguments, layouts and errors as for attn_decode_splitkv
+ * ------------------------------------------------------------------------------------------ */
+ATTN_API size_t attn_decode_multi_workspace_bytes(attn_dims_t dims, int Tmax, int n_q, int num_splits);
+ATTN_API attn_status_t attn_decode_multi(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax, int n_q,
+                                attn_dims_t dims, int num_splits, void* o, float* lse, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * attn_decode_paged — attn_decode_splitkv over a paged KV cache.
  *
  * [COOPT] Opt-Pa: sequences are cut into fixed-size pages (e.g. 512 tokens) and only pages that

@@ -103,6 +103,29 @@ def decode(q, k, v, kv_lens, *, scale: float, k_scale=None, v_scale=None):
     return o[:, 0], lse[:, :, 0]
 
 
+def decode_multi(q, k, v, kv_lens, *, scale: float, k_scale=None, v_scale=None):
+    """Multi-token decode: the cache already holds the n_q new tokens, so token i of sequence b
+    is at position len_b - n_q + i (past length + index among the new tokens, as the ORT GQA
+    analysis positions packed tokens, "Code analysis 4") and attends causally to the cache.
+
+    q: [B, n_q, Hq, D]; k, v: [B, Tmax, Hkv, D]; kv_lens [B].
+    Returns (o [B, n_q, Hq, D], lse [B, n_q, Hq]).
+    """
+    q = as_f64(q)
+    B, n_q, Hq, D = q.shape
+    lens = [int(x) for x in np.asarray(kv_lens).reshape(-1)]
+    o = np.zeros((B, n_q, Hq, D))
+    lse = np.full((B, n_q, Hq), -np.inf)
+    for b in range(B):
+        ks = None if k_scale is None else k_scale[b:b + 1]
+        vs = None if v_scale is None else v_scale[b:b + 1]
+        ob, lb = attention(q[b:b + 1], k[b:b + 1], v[b:b + 1], scale=scale, causal=True, q_pos0=lens[b] - n_q,
+                           kv_pos0=0, kv_lens=[lens[b]], k_scale=ks, v_scale=vs)
+        o[b] = ob[0]
+        lse[b] = np.asarray(lb[0]).T
+    return o, lse
+
+
 def merge_lse(o_parts, lse_parts):
     """Exact merge of partial attention results over disjoint key sets.
 

@@ -113,6 +113,26 @@ def test_decode_paged_invalid_args(L, case):
     assert st == 1
 
 
+@pytest.mark.parametrize("case", [dict(n_q=0), dict(q=None), dict(k=None), dict(kv_dtype=1), dict(ws=None)])
+def test_decode_multi_invalid_args(L, case):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, kv_dtype=0, k_scale=None, v_scale=None, kv_lens=FAKE, Tmax=4096, n_q=2,
+             dims=_dims(D=128), num_splits=4, o=FAKE, lse=None, ws=FAKE, ws_bytes=1 << 30)
+    a.update(case)
+    st = L.attn_decode_multi(a["q"], a["k"], a["v"], a["kv_dtype"], a["k_scale"], a["v_scale"], a["kv_lens"],
+                             a["Tmax"], a["n_q"], a["dims"], a["num_splits"], a["o"], a["lse"], a["ws"], a["ws_bytes"],
+                             None)
+    assert st == 1
+
+
+def test_decode_multi_rows_beyond_the_mma(L):
+    # 4 tokens x a group of 8 heads = 32 rows > 16
+    st = L.attn_decode_multi(FAKE, FAKE, FAKE, 0, None, None, FAKE, 4096, 4, _dims(Hq=32, Hkv=4, D=128), 4, FAKE,
+                             None, FAKE, 1 << 30, None)
+    assert st == 2
+    d = _dims(B=4, Hq=32, Hkv=8, D=128)
+    assert L.attn_decode_multi_workspace_bytes(d, 8192, 3, 4) == 3 * L.attn_decode_workspace_bytes(d, 8192, 4) - 2 * 256
+
+
 def test_decode_workspace_and_splits(L):
     d = _dims(B=4, Hq=32, Hkv=8, D=128)
     for P in (1, 2, 7, 19):
