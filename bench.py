@@ -349,6 +349,43 @@ def bench_decode(name, steps, warmup, world, dev, pk, paged=False, n_q=1):
             "launches": steps * (2 if splits > 1 else 1)}
 
 
+VARLEN = "prefill_varlen_b16_h32g8_d128_ragged512_2048"
+
+
+def bench_prefill_varlen(steps, warmup, world, dev, pk):
+    """Packed variable-length causal prefill (attn_prefill_varlen), inputs resident on the device."""
+    from exact_long_context_tmem_b200 import attn as A
+
+    w = I.WORKLOADS[VARLEN]
+    d = I.varlen_inputs(w)
+    qd, kd, vd, cu = d["q"].to(dev), d["k"].to(dev), d["v"].to(dev), d["cu"].to(dev)
+    max_s = int(d["lens"].max())
+    o = torch.empty_like(qd)
+    lse = torch.empty((qd.shape[0], w.Hq), dtype=torch.float32, device=dev)
+
+    def step():
+        A.attn_prefill_varlen(qd, kd, vd, cu, cu, max_s, causal=True, o=o, lse=lse)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    flops = sum(4.0 * w.D * w.Hq * int(n) * (int(n) + 1) / 2 for n in d["lens"])
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": VARLEN, "value": round(tf * world, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "tokens": int(d["lens"].sum()), "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / pk["bf16_tflops"], 4), "traffic": None}, "launches": steps}
+
+
 def bench_stream(dev, pk):
     from exact_long_context_tmem_b200 import attn as A
 
@@ -409,7 +446,8 @@ def main():
     ap.add_argument("--stream", action="store_true", help="also run the 1M-token streamed prefill")
     ap.add_argument("--cpu-rows", type=int, default=128)
     ap.add_argument("--workloads",
-                    default="prefill,decode_bf16,decode_fp8,decode_bf16_paged,decode_fp8_paged,decode_bf16_multi,decode_fp8_multi",
+                    default="prefill,prefill_varlen,decode_bf16,decode_fp8,decode_bf16_paged,decode_fp8_paged,"
+                            "decode_bf16_multi,decode_fp8_multi",
                     help="comma list of prefill, decode_bf16, decode_fp8 (profiling runs select one)")
     args = ap.parse_args()
     w = I.WORKLOADS[HEADLINE]
@@ -460,6 +498,7 @@ def main():
                 dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk, paged=True))
             if key + "_multi" in sel:
                 dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk, n_q=4))
+    varlen = bench_prefill_varlen(args.steps, args.warmup, world, dev, pk) if "prefill_varlen" in sel else None
     st, site = A.attn_device_status(reset=True)
     if st != 0:
         raise SystemExit(f"device status {st} at wait site {site}")
@@ -467,7 +506,7 @@ def main():
     cpu = None
     if pre is None:
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "partial": True, "decode": dec}), flush=True)
+            print(json.dumps({"metric": METRIC, "partial": True, "decode": dec, "prefill_varlen": varlen}), flush=True)
         return
     if rank == 0 and world == 1:
         tf, dt, rows = oracle_sample(w, args.cpu_rows)
@@ -479,7 +518,7 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic N(0,1), seeded", "config": config, "roofline": pre["roofline"],
                 "cpu_baseline": cpu, "e2e": pre["e2e"], "clocks": pre["clocks"], "gpu_launches": pre["launches"],
-                "decode": dec, "stream": stream}
+                "decode": dec, "prefill_varlen": varlen, "stream": stream}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -7,7 +7,7 @@ Importing the package does not load the library; the first call does, and fails 
 if it is missing.
 """
 
-_API = ("attn_prefill", "attn_decode_splitkv", "attn_decode_splitkv_noalloc", "attn_decode_paged", "attn_decode_multi", "attn_decode_workspace_bytes", "attn_decode_num_splits",
+_API = ("attn_prefill", "attn_decode_splitkv", "attn_decode_splitkv_noalloc", "attn_decode_paged", "attn_prefill_varlen", "attn_decode_multi", "attn_decode_workspace_bytes", "attn_decode_num_splits",
         "attn_merge_lse", "attn_chunked_stream", "attn_stream_plan", "attn_stream_task", "attn_device_status",
         "attn_set_wait_limit_ns", "attn_debug_wait_probe", "attn_debug_inject", "attn_status_string", "AttnError")
 

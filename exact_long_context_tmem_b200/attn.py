@@ -25,7 +25,7 @@ ATTN_BF16, ATTN_FP8_E4M3, ATTN_F32 = 0, 1, 2
 
 EXPORTS = [
     "attn_prefill", "attn_decode_workspace_bytes", "attn_decode_num_splits", "attn_decode_splitkv",
-    "attn_decode_splitkv_noalloc", "attn_decode_paged", "attn_decode_multi", "attn_decode_multi_workspace_bytes",
+    "attn_decode_splitkv_noalloc", "attn_decode_paged", "attn_prefill_varlen", "attn_decode_multi", "attn_decode_multi_workspace_bytes",
     "attn_merge_lse", "attn_stream_plan", "attn_stream_task", "attn_chunked_stream", "attn_status_string",
     "attn_last_cuda_error", "attn_device_status", "attn_set_wait_limit_ns", "attn_debug_wait_probe",
     "attn_debug_inject", "attn_debug_exp2",
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
     L.attn_decode_splitkv_noalloc.restype = i
     L.attn_decode_paged.argtypes = [vp, vp, vp, i, vp, vp, vp, i, i, i, vp, Dims, i, vp, vp, vp, sz, vp]
     L.attn_decode_paged.restype = i
+    L.attn_prefill_varlen.argtypes = [vp, vp, vp, vp, i, vp, Dims, vp, vp, i, i, i, i, vp]
+    L.attn_prefill_varlen.restype = i
     L.attn_decode_multi_workspace_bytes.argtypes = [Dims, i, i, i]
     L.attn_decode_multi_workspace_bytes.restype = sz
     L.attn_decode_multi.argtypes = [vp, vp, vp, i, vp, vp, vp, i, i, Dims, i, vp, vp, vp, sz, vp]
@@ -183,6 +185,28 @@ def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: 
                                    _ptr(v_scale), _ptr(kv_lens), int(Tmax), dims, int(num_splits), _ptr(o),
                                    _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, *, causal: bool = True,
+                        scale: float | None = None, o=None, lse=None, want_lse: bool = True,
+                        out_dtype=torch.bfloat16, stream=None):
+    """Packed batch: q [total_q,Hq,D], k/v [total_k,Hkv,D] bf16; cu_seqlens_q/k int32 [B+1] on the
+    device -> (o [total_q,Hq,D], lse [total_q,Hq] float32)."""
+    _need_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if o is None:
+        o = torch.empty((total_q, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((total_q, Hq), dtype=torch.float32, device=q.device)
+    od = ATTN_F32 if o.dtype == torch.float32 else ATTN_BF16
+    st = lib().attn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), od, _ptr(lse), _dims(B, Hq, Hkv, D, scale),
+                                   _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(total_q), int(total_k),
+                                   int(max_seqlen_q), int(bool(causal)), _stream(stream))
+    _check(st, "attn_prefill_varlen")
     return o, lse
 
 

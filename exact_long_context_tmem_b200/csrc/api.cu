@@ -94,17 +94,22 @@ static constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- prefill
 
+// Dense batch: q [B, S, Hq, D], k/v [B, T, Hkv, D].  Packed batch (cu_q non-null): q/o/lse rows
+// [total_q] and k/v rows [total_k] (S = total_q, T = total_k, a single TMA batch), the sequences
+// cut by the device cumulative lengths, and max_s the longest query count (grid size).
 template <int D>
 static attn_status_t launch_prefill(const void* q, const void* k, const void* v, void* o, int o_f32, float* lse,
                                     const attn_dims_t& d, int S, int T, int causal, long long q_pos0,
-                                    long long kv_pos0, cudaStream_t stream) {
+                                    long long kv_pos0, cudaStream_t stream, const int* cu_q = nullptr,
+                                    const int* cu_k = nullptr, int max_s = 0) {
   using C = PrefillCfg<D>;
   static std::atomic<uint64_t> smem_done{0};
   attn_status_t st = ensure_smem(prefill_fwd_sm100<D>, C::SMEM_BYTES, smem_done);
   if (st != ATTN_OK) return st;
   CUtensorMap mq, mk, mv;
-  const uint64_t dq[4] = {(uint64_t)D, (uint64_t)d.Hq, (uint64_t)S, (uint64_t)d.B};
-  const uint64_t dk[4] = {(uint64_t)D, (uint64_t)d.Hkv, (uint64_t)T, (uint64_t)d.B};
+  const uint64_t nb = cu_q ? 1 : (uint64_t)d.B;
+  const uint64_t dq[4] = {(uint64_t)D, (uint64_t)d.Hq, (uint64_t)std::max(S, 1), nb};
+  const uint64_t dk[4] = {(uint64_t)D, (uint64_t)d.Hkv, (uint64_t)std::max(T, 1), nb};
   const uint32_t box[4] = {64, 1, 128, 1};
   if ((st = make_map_4d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dq, box)) != ATTN_OK) return st;
   if ((st = make_map_4d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box)) != ATTN_OK) return st;
@@ -121,7 +126,7 @@ static attn_status_t launch_prefill(const void* q, const void* k, const void* v,
   p.q_pos0 = q_pos0;
   p.kv_pos0 = kv_pos0;
   p.scale_log2 = d.scale * kLog2e;
-  p.n_qtiles = (S + 127) / 128;
+  p.n_qtiles = ((cu_q ? max_s : S) + 127) / 128;
   p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
   p.n_head_units = p.pair_heads ? d.Hq / 2 : d.Hq;
   p.n_q_units = p.pair_heads ? p.n_qtiles : (p.n_qtiles + 1) / 2;
@@ -131,6 +136,9 @@ static attn_status_t launch_prefill(const void* q, const void* k, const void* v,
   p.o = o;
   p.o_f32 = o_f32;
   p.lse = lse;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  if (p.n_items == 0) return ATTN_OK;
   prefill_fwd_sm100<D><<<p.n_items, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   ATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
@@ -181,23 +189,23 @@ static size_t decode_ws_bytes(const attn_dims_t& d, int P, int n_q = 1) {
   return rows * d.D * sizeof(float) + rows * sizeof(float) + 256;
 }
 
-template <bool FP8, int GP>
+template <bool FP8, int GP, bool MULTI>
 static attn_status_t launch_decode_gp(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p,
                                       dim3 grid, cudaStream_t stream) {
   static std::atomic<uint64_t> smem_done{0};
   if (FP8) {
-    attn_status_t st = ensure_smem(decode_fp8_sm100<GP>, DecodeFp8Cfg<GP>::SMEM_BYTES, smem_done);
+    attn_status_t st = ensure_smem(decode_fp8_sm100<GP, MULTI>, DecodeFp8Cfg<GP>::SMEM_BYTES, smem_done);
     if (st != ATTN_OK) return st;
     // Persistent: one CTA per SM (at most one per work item), each walking items c, c + grid, ...
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long items = (long long)grid.x * grid.y * grid.z;
     const dim3 pgrid((unsigned)std::min<long long>(items, std::max(sms, 1)));
-    decode_fp8_sm100<GP><<<pgrid, DecodeFp8Cfg<GP>::THREADS, DecodeFp8Cfg<GP>::SMEM_BYTES, stream>>>(mk, mv, p);
+    decode_fp8_sm100<GP, MULTI><<<pgrid, DecodeFp8Cfg<GP>::THREADS, DecodeFp8Cfg<GP>::SMEM_BYTES, stream>>>(mk, mv, p);
   } else {
-    attn_status_t st = ensure_smem(decode_split_sm100<GP>, DecodeCfg::SMEM_BYTES, smem_done);
+    attn_status_t st = ensure_smem(decode_split_sm100<GP, MULTI>, DecodeCfg::SMEM_BYTES, smem_done);
     if (st != ATTN_OK) return st;
-    decode_split_sm100<GP><<<grid, DecodeCfg::THREADS, DecodeCfg::SMEM_BYTES, stream>>>(mk, mv, p);
+    decode_split_sm100<GP, MULTI><<<grid, DecodeCfg::THREADS, DecodeCfg::SMEM_BYTES, stream>>>(mk, mv, p);
   }
   ATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
@@ -259,11 +267,19 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   if ((long long)P * d.Hkv * d.B > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;  // work items are int-indexed
   // The query group is padded to the next power of two (<= 16) so the kernels' per-row loops unroll.
   const int R = p.G * n_q;  // MMA rows of one (sequence, KV head)
-  if (R <= 1) st = launch_decode_gp<FP8, 1>(mk, mv, p, grid, stream);
-  else if (R <= 2) st = launch_decode_gp<FP8, 2>(mk, mv, p, grid, stream);
-  else if (R <= 4) st = launch_decode_gp<FP8, 4>(mk, mv, p, grid, stream);
-  else if (R <= 8) st = launch_decode_gp<FP8, 8>(mk, mv, p, grid, stream);
-  else st = launch_decode_gp<FP8, 16>(mk, mv, p, grid, stream);
+  // Single-token decode runs instances without per-row key limits (one compare per token).
+  if (n_q == 1) {
+    if (R <= 1) st = launch_decode_gp<FP8, 1, false>(mk, mv, p, grid, stream);
+    else if (R <= 2) st = launch_decode_gp<FP8, 2, false>(mk, mv, p, grid, stream);
+    else if (R <= 4) st = launch_decode_gp<FP8, 4, false>(mk, mv, p, grid, stream);
+    else if (R <= 8) st = launch_decode_gp<FP8, 8, false>(mk, mv, p, grid, stream);
+    else st = launch_decode_gp<FP8, 16, false>(mk, mv, p, grid, stream);
+  } else {
+    if (R <= 2) st = launch_decode_gp<FP8, 2, true>(mk, mv, p, grid, stream);
+    else if (R <= 4) st = launch_decode_gp<FP8, 4, true>(mk, mv, p, grid, stream);
+    else if (R <= 8) st = launch_decode_gp<FP8, 8, true>(mk, mv, p, grid, stream);
+    else st = launch_decode_gp<FP8, 16, true>(mk, mv, p, grid, stream);
+  }
   if (st != ATTN_OK) return st;
   if (P > 1) {
     MergeParams mp{};
@@ -362,6 +378,42 @@ attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o,
   const int f32 = o_dtype == ATTN_F32;
   if (dims.D == 128) return launch_prefill<128>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st);
   return launch_prefill<64>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st);
+}
+
+attn_status_t attn_prefill_varlen(const void* q, const void* k, const void* v, void* o, attn_dtype_t o_dtype,
+                                  float* lse, attn_dims_t dims, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                  int total_q, int total_k, int max_seqlen_q, int causal, void* stream) {
+  if (!dims_ok(dims) || total_q < 0 || total_k < 0 || max_seqlen_q < 0) return ATTN_ERR_INVALID_ARG;
+  if (o_dtype != ATTN_BF16 && o_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  if (dims.B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+  if (!q || !o || !cu_seqlens_q || !cu_seqlens_k || (total_k > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || (total_k > 0 && (!aligned16(k) || !aligned16(v))) ||
+      (lse && !aligned4(lse)) || !aligned4(cu_seqlens_q) || !aligned4(cu_seqlens_k))
+    return ATTN_ERR_INVALID_ARG;
+  if (dims.D != 64 && dims.D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (total_k == 0) {  // no keys anywhere: every row is empty (O = 0, LSE = -inf)
+    MergeParams mp{};
+    mp.P = 0;
+    mp.R = (long long)total_q * dims.Hq;
+    mp.o_out = o;
+    mp.o_f32 = o_dtype == ATTN_F32;
+    mp.lse_out = lse;
+    mp.accumulate = 0;
+    const long long blocks = (mp.R + 7) / 8;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dims.D == 128) merge_lse_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(mp);
+    else merge_lse_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(mp);
+    ATTN_CUDA(cudaGetLastError());
+    return ATTN_OK;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int f32 = o_dtype == ATTN_F32;
+  if (dims.D == 128)
+    return launch_prefill<128>(q, k, v, o, f32, lse, dims, total_q, total_k, causal, 0, 0, st, cu_seqlens_q,
+                               cu_seqlens_k, max_seqlen_q);
+  return launch_prefill<64>(q, k, v, o, f32, lse, dims, total_q, total_k, causal, 0, 0, st, cu_seqlens_q,
+                            cu_seqlens_k, max_seqlen_q);
 }
 
 int attn_decode_num_splits(attn_dims_t dims, int Tmax, int num_splits) {

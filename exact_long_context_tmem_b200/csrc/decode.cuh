@@ -199,9 +199,11 @@ __device__ __forceinline__ bool decode_softmax_core(DecodeRows<GP>& rows, const 
 }
 
 // bf16 decode: the 16 S^T columns of this lane, scaled by sc (log2 domain), then the shared core.
-template <int GP, bool F16P>
+// MULTI: several query tokens share the rows, each with its own key limit rlim[g]; otherwise every
+// row's limit is t1 (kept as one compare).
+template <int GP, bool F16P, bool MULTI>
 __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j, bool has_prev, int lane, int wq,
-                                                    int t, int tok, const int (&rlim)[GP], float sc, float vs,
+                                                    int t, int tok, int t1, const int (&rlim)[GP], float sc, float vs,
                                                     uint32_t tS_lane,
                                                     uint32_t tO_lane, float* red_max, uint64_t* red_bar,
                                                     uint64_t* prev_pv, uint32_t prev_pv_parity, uint8_t* p_tile,
@@ -211,7 +213,8 @@ __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j,
   tmem_wait_ld();
   float x[GP];
 #pragma unroll
-  for (int g = 0; g < GP; ++g) x[g] = tok < rlim[g] ? __uint_as_float(sv[g]) * sc : -INFINITY;
+  for (int g = 0; g < GP; ++g)
+    x[g] = (MULTI ? tok < rlim[g] : tok < t1) ? __uint_as_float(sv[g]) * sc : -INFINITY;
   return decode_softmax_core<GP, F16P>(rows, x, j, has_prev, lane, wq, t, vs, tO_lane, red_max, red_bar, prev_pv,
                                        prev_pv_parity, p_tile, threshold);
 }
@@ -222,7 +225,7 @@ __device__ __forceinline__ bool decode_softmax_tile(DecodeRows<GP>& rows, int j,
 // a per-tile barrier two phases can still be pending here, and a parity wait could be satisfied
 // by the older one.  sum_parity is the phase of sum_bar; o_free (if not null) is arrived on once
 // O^T has been read, so the accumulator can take the next split.
-template <int GP>
+template <int GP, bool MULTI>
 __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const DecodeParams& p, int G, int split,
                                                 int kvh, int b, int lane, int wq, int t, uint32_t tO_lane,
                                                 float* red_sum, uint64_t* sum_bar, uint32_t sum_parity,
@@ -254,7 +257,7 @@ __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const Deco
       const float ov = (l > 0.f) ? __uint_as_float(orow[g]) / l : 0.f;
       const float lse = (l > 0.f) ? (rows.m_used[g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (g == t) my_lse = lse;
-      const long long h = decode_row_index(p, b, kvh, g);
+      const long long h = MULTI ? decode_row_index(p, b, kvh, g) : (long long)b * p.Hq + (long long)kvh * p.G + g;
       if (p.n_splits == 1) {
         p.o[h * D + t] = __float2bfloat16_rn(ov);
       } else {
@@ -263,7 +266,7 @@ __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const Deco
     }
   }
   if (t < R) {
-    const long long h = decode_row_index(p, b, kvh, t);
+    const long long h = MULTI ? decode_row_index(p, b, kvh, t) : (long long)b * p.Hq + (long long)kvh * p.G + t;
     if (p.n_splits == 1) {
       if (p.lse) p.lse[h] = my_lse;
     } else {
@@ -336,7 +339,7 @@ __device__ __forceinline__ void convert_row_e4m3(const uint8_t* codes_tile, uint
   }
 }
 
-template <int GP>
+template <int GP, bool MULTI>
 __global__ void __launch_bounds__(192, 1)
     decode_split_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const DecodeParams p) {
@@ -521,7 +524,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       // PV(j-1) is the j-th completion of o_ready; S(j) completing implies PV(j-2) done, so at
       // most one phase is pending and the parity wait is unambiguous.
-      if (!(ok = decode_softmax_tile<GP, false>(rows, j, j > 0, lane, wq, t, tok, rlim, p.scale_log2, 1.f,
+      if (!(ok = decode_softmax_tile<GP, false, MULTI>(rows, j, j > 0, lane, wq, t, tok, t1, rlim, p.scale_log2, 1.f,
                                                 tS0 + (j & 1) * 16 + lane_off, tO + lane_off, red_max, red_bar,
                                                 o_ready, (j - 1) & 1, smem + C::OFF_P + (j & 1) * C::P_BYTES,
                                                 C::RESCALE_THRESHOLD)))
@@ -542,7 +545,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(&p_full[j & 1]);
     }
     if (ok)
-      decode_epilogue<GP>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, 0, o_final, 0,
+      decode_epilogue<GP, MULTI>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, 0, o_final, 0,
                           nullptr);
   }
   tc_fence_before();

@@ -239,9 +239,9 @@ __device__ __forceinline__ uint32_t p8_offset(int r, int t) {
 // E4M3 pieces into P^T.  j counts this warpgroup's tiles (phases of red_bar); has_prev says O^T
 // already holds earlier tiles of the item; prev_pv / prev_pv_parity name the unambiguous phase
 // that completes with the previous PV.  Returns false, warp-uniformly, if a bounded wait ran out.
-template <int GP, int NQ, int NP, int NS>
+template <int GP, int NQ, int NP, int NS, bool MULTI>
 __device__ __forceinline__ bool fp8_softmax_tile(DecodeRows<GP>& rows, int j, bool has_prev, int lane, int wq, int t,
-                                                 int tok, const int (&rlim)[GP], float sck, float vs,
+                                                 int tok, int t1, const int (&rlim)[GP], float sck, float vs,
                                                  const float (&fq)[GP],
                                                  uint32_t tS_lane, uint32_t tO_lane, float* red_max,
                                                  uint64_t* red_bar, uint64_t* s_free, uint64_t* pv_done,
@@ -256,7 +256,7 @@ __device__ __forceinline__ bool fp8_softmax_tile(DecodeRows<GP>& rows, int j, bo
   for (int g = 0; g < GP; ++g) {
     const float s12 = fmaf(__uint_as_float(sv[2 * GP + g]), 0.0625f, __uint_as_float(sv[GP + g]));
     const float s = fmaf(s12, 0.0625f, __uint_as_float(sv[g]));
-    x[g] = tok < rlim[g] ? s * (sck * fq[g]) : -INFINITY;
+    x[g] = (MULTI ? tok < rlim[g] : tok < t1) ? s * (sck * fq[g]) : -INFINITY;
     y[g] = x[g] + lv;
   }
   float* rm = red_max + (j & 1) * 64;
@@ -321,7 +321,7 @@ __device__ __forceinline__ bool fp8_softmax_tile(DecodeRows<GP>& rows, int j, bo
 // (o_full, phase o_parity), read O^T (then release it through o_free), and thread t (= output
 // element d) writes o[g][t] = (sum over pieces k of O^T[t][k GP + g] / 16^k) / l_g and, for t < G,
 // lse_t = ln 2 (m_g + log2 l_g).
-template <int GP, int NP>
+template <int GP, int NP, bool MULTI>
 __device__ __forceinline__ bool fp8_epilogue(DecodeRows<GP>& rows, const DecodeParams& p, int G, int split, int kvh,
                                              int b, int lane, int wq, int t, uint32_t tO_lane, float* red_sum,
                                              uint64_t* sum_bar, uint32_t sum_parity, uint64_t* o_full,
@@ -353,7 +353,7 @@ __device__ __forceinline__ bool fp8_epilogue(DecodeRows<GP>& rows, const DecodeP
       const float ov = (l > 0.f) ? acc / l : 0.f;
       const float lse = (l > 0.f) ? (rows.m_used[g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (g == t) my_lse = lse;
-      const long long h = decode_row_index(p, b, kvh, g);
+      const long long h = MULTI ? decode_row_index(p, b, kvh, g) : (long long)b * p.Hq + (long long)kvh * p.G + g;
       if (p.n_splits == 1) {
         p.o[h * D + t] = __float2bfloat16_rn(ov);
       } else {
@@ -362,7 +362,7 @@ __device__ __forceinline__ bool fp8_epilogue(DecodeRows<GP>& rows, const DecodeP
     }
   }
   if (t < R) {
-    const long long h = decode_row_index(p, b, kvh, t);
+    const long long h = MULTI ? decode_row_index(p, b, kvh, t) : (long long)b * p.Hq + (long long)kvh * p.G + t;
     if (p.n_splits == 1) {
       if (p.lse) p.lse[h] = my_lse;
     } else {
@@ -372,7 +372,7 @@ __device__ __forceinline__ bool fp8_epilogue(DecodeRows<GP>& rows, const DecodeP
   return true;
 }
 
-template <int GP>
+template <int GP, bool MULTI>
 __global__ void __launch_bounds__(256, 1)
     decode_fp8_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
@@ -734,7 +734,8 @@ __global__ void __launch_bounds__(256, 1)
         if (!(ok = mbar_wait_warp(&s_full[bs], (j / NS) & 1, SITE_DC_SM_S))) break;
         if (t == 0) ATTN_EVT(j, 4);
         tc_fence_after();
-        if (!(ok = fp8_softmax_tile<GP, NQ, NP, NS>(rows, j, l > 0, lane, wq, t, tok, rlim, p.scale_log2 * ks, vs, fq,
+        if (!(ok = fp8_softmax_tile<GP, NQ, NP, NS, MULTI>(rows, j, l > 0, lane, wq, t, tok, cur.t1, rlim,
+                                                           p.scale_log2 * ks, vs, fq,
                                                     tS0 + bs * NQ + lane_off, tO, red_max, red_bar, s_free, pv_done,
                                                     smem + C::OFF_P + bs * C::P_BYTES, C::RESCALE_THRESHOLD)))
           break;
@@ -744,7 +745,7 @@ __global__ void __launch_bounds__(256, 1)
         if (t == 0) ATTN_EVT(j, 5);
       }
       if (!ok) break;
-      ok = fp8_epilogue<GP, NP>(rows, p, G, cur.split, cur.kvh, cur.b, lane, wq, t, tO, red_sum, sum_bar, ie & 1,
+      ok = fp8_epilogue<GP, NP, MULTI>(rows, p, G, cur.split, cur.kvh, cur.b, lane, wq, t, tO, red_sum, sum_bar, ie & 1,
                                 &o_full[ie & 1], (ie >> 1) & 1, &o_free[ie & 1]);
       ++ie;
       cur = nxt;

@@ -41,6 +41,12 @@ struct PrefillParams {
   void* o;
   int o_f32;
   float* lse;
+  // Packed variable-length batch (ORT packed-QSA analysis, "Code analysis": cumulative sequence
+  // lengths, and a token's position = past length + its index among the new tokens): sequence b's
+  // queries are rows cu_q[b] .. cu_q[b+1]-1 of q/o/lse and its keys rows cu_k[b] .. cu_k[b+1]-1 of
+  // k/v; query i sits at position (len_k - len_q) + i, key j at j.  Null for a dense batch.
+  const int* cu_q;
+  const int* cu_k;
 };
 
 template <int D>
@@ -67,6 +73,10 @@ struct PrefillItem {
   bool active[2];
   int n_tiles;
   int kvh;
+  int S, T;                    // this sequence's query and key counts
+  long long q_pos0, kv_pos0;   // absolute positions of its query row 0 and key 0
+  int q_base, k_base, bc;      // TMA token offsets of its rows 0 and batch coordinate
+  long long o_row0;            // row of query 0 in o / lse (rows of Hq heads)
 };
 
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int idx) {
@@ -76,6 +86,27 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
   const int rem = idx % per_q;
   it.b = rem / p.n_head_units;
   const int hunit = rem % p.n_head_units;
+  if (p.cu_q) {
+    const int qs = __ldg(p.cu_q + it.b), qe = __ldg(p.cu_q + it.b + 1);
+    const int ks = __ldg(p.cu_k + it.b), ke = __ldg(p.cu_k + it.b + 1);
+    it.S = qe > qs ? qe - qs : 0;
+    it.T = ke > ks ? ke - ks : 0;
+    it.q_pos0 = (long long)it.T - it.S;  // the queries are the sequence's last S tokens
+    it.kv_pos0 = 0;
+    it.q_base = qs;
+    it.k_base = ks;
+    it.bc = 0;
+    it.o_row0 = qs;
+  } else {
+    it.S = p.S;
+    it.T = p.T;
+    it.q_pos0 = p.q_pos0;
+    it.kv_pos0 = p.kv_pos0;
+    it.q_base = 0;
+    it.k_base = 0;
+    it.bc = it.b;
+    it.o_row0 = (long long)it.b * p.S;
+  }
   for (int s = 0; s < 2; ++s) {
     int head, qt;
     if (p.pair_heads) {
@@ -87,16 +118,16 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
     }
     it.head[s] = head;
     it.q_lo[s] = qt * 128;
-    it.active[s] = it.q_lo[s] < p.S;
+    it.active[s] = it.q_lo[s] < it.S;
   }
   it.kvh = it.head[0] / p.G;
   int n = 0;
   for (int s = 0; s < 2; ++s) {
     if (!it.active[s]) continue;
-    long long kv_end = p.T;
+    long long kv_end = it.T;
     if (p.causal) {
-      const long long q_last = (long long)min(p.S, it.q_lo[s] + 128) - 1;
-      long long e = p.q_pos0 + q_last - p.kv_pos0 + 1;
+      const long long q_last = (long long)min(it.S, it.q_lo[s] + 128) - 1;
+      long long e = it.q_pos0 + q_last - it.kv_pos0 + 1;
       kv_end = e < kv_end ? e : kv_end;
     }
     if (kv_end < 0) kv_end = 0;
@@ -170,8 +201,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
       for (int s = 0; s < 2; ++s)
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(sQ + s * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, q_full, bx * 64, it.head[s], it.q_lo[s],
-                      it.b);
+          tma_load_4d(sQ + s * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, q_full, bx * 64, it.head[s],
+                      it.q_base + it.q_lo[s], it.bc);
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < n && ok; ++j) {
@@ -182,13 +213,13 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem + C::OFF_K + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmK, &k_full[st], bx * 64, it.kvh,
-                      j * 128, it.b);
+                      it.k_base + j * 128, it.bc);
         ATTN_TRACE_AT(0, 5, j);
         if (!mbar_wait(&v_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; issued = 2 * j + 1; break; }
         mbar_arrive_expect_tx(&v_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem + C::OFF_V + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmV, &v_full[st], bx * 64, it.kvh,
-                      j * 128, it.b);
+                      it.k_base + j * 128, it.bc);
         issued = 2 * j + 2;
       }
       ATTN_TRACE_AT(0, 6, issued);
@@ -295,7 +326,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem + slot * 128 + lane_off;
     const uint32_t tO = tmem + 256 + slot * D + lane_off;
     const int q_lo = it.q_lo[slot];
-    const long long rel = p.q_pos0 + q_lo + r - p.kv_pos0;  // key index limit (inclusive) for causal
+    const long long rel = it.q_pos0 + q_lo + r - it.kv_pos0;  // key index limit (inclusive) for causal
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -306,7 +337,7 @@ __global__ void __launch_bounds__(384, 1)
       if (r == 0) ATTN_EVT(j, slot * 8 + 1);
       tc_fence_after();
       const int kv0 = j * 128;
-      long long lim64 = (long long)p.T - kv0;  // column c is a visible key iff c < lim
+      long long lim64 = (long long)it.T - kv0;  // column c is a visible key iff c < lim
       if (p.causal) {
         const long long c2 = rel + 1 - kv0;
         lim64 = c2 < lim64 ? c2 : lim64;
@@ -391,7 +422,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     // ---- epilogue: O / l -> global, LSE = ln2 * (m + log2 l)
     const int row = q_lo + r;
-    const bool row_ok = it.active[slot] && row < p.S;
+    const bool row_ok = it.active[slot] && row < it.S;
     const bool have_o = n > 0;
     if (r == 0) ATTN_TRACE_AT(4 + slot, 1, ok);
     if (ok && have_o) {
@@ -401,7 +432,7 @@ __global__ void __launch_bounds__(384, 1)
     if (r == 0) ATTN_TRACE_AT(4 + slot, 2, ok);
     if (ok) {
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const long long orow = (((long long)it.b * p.S + row) * p.Hq + it.head[slot]) * D;
+      const long long orow = ((it.o_row0 + row) * p.Hq + it.head[slot]) * D;
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
         if (have_o) {  // warp-collective load for every lane; only rows < S are stored
@@ -433,7 +464,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (p.lse && row_ok) {
         const float lse = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        p.lse[((long long)it.b * p.S + row) * p.Hq + it.head[slot]] = lse;
+        p.lse[(it.o_row0 + row) * p.Hq + it.head[slot]] = lse;
       }
     }
   }

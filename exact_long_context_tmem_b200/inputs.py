@@ -56,6 +56,9 @@ WORKLOADS = {
     "decode_fp8_b16_h32g8_d128_t32768": Workload(
         "decode_fp8_b16_h32g8_d128_t32768", "decode", B=16, Hq=32, Hkv=8, D=128,
         len_lo=32768, len_hi=32768, kv_fp8=True, seed=1003),
+    "prefill_varlen_b16_h32g8_d128_ragged512_2048": Workload(
+        "prefill_varlen_b16_h32g8_d128_ragged512_2048", "prefill_varlen", B=16, Hq=32, Hkv=8, D=128,
+        len_lo=512, len_hi=2048, seed=1005),
     "stream_b1_h32g8_d128_s1m_chunk64k": Workload(
         "stream_b1_h32g8_d128_s1m_chunk64k", "stream", B=1, Hq=32, Hkv=8, D=128,
         S=1 << 20, T=1 << 20, chunk_tokens=65536, budget_bytes=16 * 10**9, seed=1004),
@@ -160,6 +163,21 @@ def decode_inputs(w: Workload, B: int | None = None, Tmax: int | None = None, se
         vf[pad] = pad_value
         out.update(k=kf, v=vf)
     return out
+
+
+def varlen_inputs(w: Workload, seed: int | None = None):
+    """Packed batch of w.B sequences, each with U{len_lo..len_hi} tokens (queries = keys: plain
+    causal prefill).  Returns q [total, Hq, D], k, v [total, Hkv, D] bf16, lengths int32 [B] and
+    cumulative lengths cu int32 [B + 1]; Q, K, V are drawn in that order, then the lengths."""
+    g = generator(w.seed if seed is None else seed)
+    lens = torch.randint(w.len_lo, w.len_hi + 1, (w.B,), generator=g, dtype=torch.int64)
+    total = int(lens.sum())
+    q = randn_bf16((total, w.Hq, w.D), g)
+    k = randn_bf16((total, w.Hkv, w.D), g)
+    v = randn_bf16((total, w.Hkv, w.D), g)
+    cu = torch.zeros(w.B + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens, 0).to(torch.int32)
+    return {"q": q, "k": k, "v": v, "lens": lens.to(torch.int32), "cu": cu}
 
 
 def paged_inputs(d: dict, page_size: int, seed: int, spare_frac: float = 0.125):

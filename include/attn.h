@@ -92,6 +92,34 @@ ATTN_API attn_status_t attn_prefill(const void* q, const void* k, const void* v,
                            long long kv_pos0, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * attn_prefill_varlen — attn_prefill over a packed batch of sequences of different lengths,
+ * with no padding.
+ *
+ * [ORT-QSA] Code analysis 1: tokens of all sequences are packed along one axis and cut by
+ * cumulative sequence lengths; a new token's position is the sequence's past length plus its
+ * index among the new tokens.  Sequence b's queries are rows cu_seqlens_q[b] ..
+ * cu_seqlens_q[b+1]-1 of q, o and lse; its keys are rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1
+ * of k and v (past tokens first, then the new ones), so query i of a sequence with Sq queries and
+ * Sk keys sits at position Sk - Sq + i and, when causal, sees keys [0, Sk - Sq + i].  Rows with no
+ * visible key get O = 0, LSE = -inf.
+ *
+ *   q, o          device [total_q, Hq, D] (q bf16; o bf16 or float32 per o_dtype)
+ *   k, v          device bf16 [total_k, Hkv, D]
+ *   lse           device float32 [total_q, Hq] or NULL
+ *   cu_seqlens_q  device int32 [B + 1], non-decreasing, cu_seqlens_q[0] = 0, cu_seqlens_q[B] = total_q
+ *   cu_seqlens_k  device int32 [B + 1], likewise ending at total_k
+ *   max_seqlen_q  the largest query count of any sequence (host value: sizes the grid; the device
+ *                 lengths are never read back)
+ *   dims.B        number of sequences; D in {64, 128}; scale as in dims
+ * Errors: ATTN_ERR_INVALID_ARG for bad sizes, null or misaligned pointers; ATTN_ERR_UNSUPPORTED for
+ * other head dims.  Cumulative lengths that break the rules above give rows with no keys, never an
+ * out-of-bounds read (TMA boxes past the packed tensors land as zeros).
+ * ------------------------------------------------------------------------------------------ */
+ATTN_API attn_status_t attn_prefill_varlen(const void* q, const void* k, const void* v, void* o, attn_dtype_t o_dtype,
+                                  float* lse, attn_dims_t dims, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                  int total_q, int total_k, int max_seqlen_q, int causal, void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * attn_decode_splitkv — one query token per sequence over a ragged KV cache.
  *
  * Flash Decoding ([ORT-CPU] Code analysis 2): the key range of each (sequence, KV head) is cut

@@ -126,6 +126,30 @@ def decode_multi(q, k, v, kv_lens, *, scale: float, k_scale=None, v_scale=None):
     return o, lse
 
 
+def prefill_varlen(q, k, v, cu_q, cu_k, *, scale: float, causal: bool):
+    """Packed variable-length prefill (ORT packed-QSA analysis, "Code analysis 1"): sequence b's
+    queries are rows cu_q[b]..cu_q[b+1]-1 of q and its keys rows cu_k[b]..cu_k[b+1]-1 of k, v; a
+    query's position is the past length (keys - queries) plus its index among the queries.
+
+    q: [total_q, Hq, D]; k, v: [total_k, Hkv, D].  Returns (o [total_q, Hq, D], lse [total_q, Hq]).
+    """
+    q = as_f64(q)
+    cu_q = [int(x) for x in np.asarray(cu_q).reshape(-1)]
+    cu_k = [int(x) for x in np.asarray(cu_k).reshape(-1)]
+    total_q, Hq, D = q.shape
+    o = np.zeros((total_q, Hq, D))
+    lse = np.full((total_q, Hq), -np.inf)
+    for b in range(len(cu_q) - 1):
+        qs, qe, ks, ke = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+        if qe <= qs:
+            continue
+        ob, lb = attention(q[None, qs:qe], k[None, ks:ke], v[None, ks:ke], scale=scale, causal=causal,
+                           q_pos0=(ke - ks) - (qe - qs), kv_pos0=0)
+        o[qs:qe] = ob[0]
+        lse[qs:qe] = np.asarray(lb[0]).T
+    return o, lse
+
+
 def merge_lse(o_parts, lse_parts):
     """Exact merge of partial attention results over disjoint key sets.
 

@@ -133,6 +133,17 @@ def test_decode_multi_rows_beyond_the_mma(L):
     assert L.attn_decode_multi_workspace_bytes(d, 8192, 3, 4) == 3 * L.attn_decode_workspace_bytes(d, 8192, 4) - 2 * 256
 
 
+@pytest.mark.parametrize("case", [dict(total_q=-1), dict(max_s=-1), dict(cu_q=None), dict(cu_k=None), dict(q=None),
+                                  dict(k=None), dict(o_dtype=1), dict(cu_q=ctypes.c_void_p(0x10002))])
+def test_prefill_varlen_invalid_args(L, case):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, o_dtype=0, lse=None, dims=_dims(D=128), cu_q=FAKE, cu_k=FAKE,
+             total_q=1000, total_k=1000, max_s=300, causal=1)
+    a.update(case)
+    st = L.attn_prefill_varlen(a["q"], a["k"], a["v"], a["o"], a["o_dtype"], a["lse"], a["dims"], a["cu_q"], a["cu_k"],
+                               a["total_q"], a["total_k"], a["max_s"], a["causal"], None)
+    assert st == 1
+
+
 def test_decode_workspace_and_splits(L):
     d = _dims(B=4, Hq=32, Hkv=8, D=128)
     for P in (1, 2, 7, 19):
