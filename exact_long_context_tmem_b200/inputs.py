@@ -36,6 +36,7 @@ class Workload:
     len_lo: int = 0  # ragged decode lengths, closed interval
     len_hi: int = 0
     kv_fp8: bool = False
+    kv_bits: int = 0  # 8 or 4: INT8 / INT4 KV cache (0: not an integer cache)
     chunk_tokens: int = 0  # streamed prefill
     budget_bytes: int = 0
     seed: int = 0
@@ -56,6 +57,12 @@ WORKLOADS = {
     "decode_fp8_b16_h32g8_d128_t32768": Workload(
         "decode_fp8_b16_h32g8_d128_t32768", "decode", B=16, Hq=32, Hkv=8, D=128,
         len_lo=32768, len_hi=32768, kv_fp8=True, seed=1003),
+    "decode_int8_b16_h32g8_d128_t32768": Workload(
+        "decode_int8_b16_h32g8_d128_t32768", "decode", B=16, Hq=32, Hkv=8, D=128,
+        len_lo=32768, len_hi=32768, kv_bits=8, seed=1006),
+    "decode_int4_b16_h32g8_d128_t32768": Workload(
+        "decode_int4_b16_h32g8_d128_t32768", "decode", B=16, Hq=32, Hkv=8, D=128,
+        len_lo=32768, len_hi=32768, kv_bits=4, seed=1007),
     "prefill_varlen_b16_h32g8_d128_ragged512_2048": Workload(
         "prefill_varlen_b16_h32g8_d128_ragged512_2048", "prefill_varlen", B=16, Hq=32, Hkv=8, D=128,
         len_lo=512, len_hi=2048, seed=1005),
@@ -122,15 +129,36 @@ def quantize_e4m3_per_token(x: torch.Tensor):
     return codes, scale.contiguous()
 
 
+def quantize_int_per_token(x: torch.Tensor, bits: int):
+    """Synthetic INT8 / INT4 KV cache: symmetric codes + one float32 scale per (batch, token,
+    head).  qmax = 127 (INT8) or 7 (INT4); scale = absmax over the head dimension / qmax (1 for
+    an all-zero row); codes = x / scale rounded half-to-even and clamped to +-qmax.  INT8 codes are
+    int8 [..., D]; INT4 codes are packed two per byte, element 2i in the low nibble of byte i and
+    element 2i+1 in the high nibble, uint8 [..., D/2].
+    """
+    qmax = {8: 127.0, 4: 7.0}[bits]
+    xf = x.float()
+    amax = xf.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / qmax, torch.ones_like(amax))
+    c = torch.round(xf / scale.unsqueeze(-1)).clamp(-qmax, qmax).to(torch.int32)
+    if bits == 8:
+        return c.to(torch.int8).contiguous(), scale.contiguous()
+    n = c & 0xF
+    packed = (n[..., 0::2] | (n[..., 1::2] << 4)).to(torch.uint8)
+    return packed.contiguous(), scale.contiguous()
+
+
 def decode_inputs(w: Workload, B: int | None = None, Tmax: int | None = None, seed: int | None = None,
                   lens: torch.Tensor | None = None, pad_value: float = float("nan")):
     """Decode workload.
 
     Returns a dict with q [B,Hq,D] bf16, kv_lens int32 [B], and either
-    k, v bf16 [B,Tmax,Hkv,D] or k_codes, v_codes uint8 [B,Tmax,Hkv,D] with
+    k, v bf16 [B,Tmax,Hkv,D] or k_codes, v_codes (uint8 E4M3 [B,Tmax,Hkv,D]; int8
+    [B,Tmax,Hkv,D] for INT8; packed uint8 [B,Tmax,Hkv,D/2] for INT4, with kv_bits) and
     k_scale, v_scale float32 [B,Tmax,Hkv].  Cache slots at or beyond a
-    sequence's length hold ``pad_value`` (NaN by default, code 0x7f for FP8),
-    so any read of padding shows up in the output.
+    sequence's length hold ``pad_value`` (NaN by default; code 0x7f for FP8 and
+    the integer caches, whose pad scales are NaN), so any read of padding shows up
+    in the output.
     """
     B = w.B if B is None else B
     g = generator(w.seed if seed is None else seed)
@@ -149,7 +177,15 @@ def decode_inputs(w: Workload, B: int | None = None, Tmax: int | None = None, se
     lens = lens.to(torch.int32)
     out = {"q": q, "kv_lens": lens, "Tmax": Tmax}
     pad = torch.arange(Tmax).unsqueeze(0) >= lens.long().unsqueeze(1)  # [B, Tmax]
-    if w.kv_fp8:
+    if w.kv_bits:
+        kc, ks = quantize_int_per_token(kf, w.kv_bits)
+        vc, vs = quantize_int_per_token(vf, w.kv_bits)
+        kc[pad] = 0x7F
+        vc[pad] = 0x7F
+        ks[pad] = pad_value
+        vs[pad] = pad_value
+        out.update(k_codes=kc, v_codes=vc, k_scale=ks, v_scale=vs, kv_bits=w.kv_bits)
+    elif w.kv_fp8:
         kc, ks = quantize_e4m3_per_token(kf)
         vc, vs = quantize_e4m3_per_token(vf)
         code_pad = 0x7F if pad_value != pad_value else 0
@@ -202,9 +238,11 @@ def paged_inputs(d: dict, page_size: int, seed: int, spare_frac: float = 0.125):
     perm = torch.randperm(total + spare, generator=g)
     table = torch.full((B, max_pages), -1, dtype=torch.int32)
     out = {"q": d["q"], "kv_lens": d["kv_lens"], "page_size": page_size, "num_pages": total + spare}
+    if "kv_bits" in d:
+        out["kv_bits"] = d["kv_bits"]
     for name in names:
         src = d[name]
-        pad_val = 0x7F if src.dtype == torch.uint8 else float("nan")
+        pad_val = 0x7F if src.dtype in (torch.uint8, torch.int8) else float("nan")
         pool = torch.full((total + spare, page_size) + tuple(src.shape[2:]), pad_val, dtype=src.dtype)
         padded = torch.full((B, max_pages * page_size) + tuple(src.shape[2:]), pad_val, dtype=src.dtype)
         padded[:, :Tmax] = src

@@ -8,6 +8,7 @@ here, and this package imports nothing from the product path.
 Modules:
   attention  exact attention rows, single-token decode, log-sum-exp merge
   fp8        E4M3 code table from the format definition
+  intq       INT8 / INT4 KV codes (two's complement, low nibble first) to values
   stream     exact-cover check of a (query block, key chunk) task list
   paged      paged KV cache: gather mapped pages into the contiguous cache, then decode
 """
