@@ -34,7 +34,10 @@ from exact_long_context_tmem_b200 import inputs as I  # noqa: E402
 
 METRIC = "prefill attn TFLOP/s & decode KV GB/s at 1 B200, as fraction of roofline"
 HEADLINE = "prefill_b2_h32g8_d128_s8192"
-DECODE_WORKLOADS = ("decode_b4_h32g8_d128_ragged64k_128k", "decode_fp8_b16_h32g8_d128_t32768")
+DECODE_WORKLOADS = (("decode_bf16", "decode_b4_h32g8_d128_ragged64k_128k"),
+                    ("decode_fp8", "decode_fp8_b16_h32g8_d128_t32768"),
+                    ("decode_int8", "decode_int8_b16_h32g8_d128_t32768"),
+                    ("decode_int4", "decode_int4_b16_h32g8_d128_t32768"))
 STREAM = "stream_b1_h32g8_d128_s1m_chunk64k"
 L2_BYTES = 126 * 10**6
 
@@ -176,8 +179,9 @@ def prefill_flops(w):
 
 def decode_bytes(w, lens):
     tok = int(lens.sum())
-    per_tok = w.Hkv * w.D * (1 if w.kv_fp8 else 2) * 2
-    if w.kv_fp8:
+    row = w.D // 2 if w.kv_bits == 4 else (w.D if (w.kv_fp8 or w.kv_bits == 8) else 2 * w.D)  # bytes per K or V row
+    per_tok = w.Hkv * row * 2
+    if w.kv_fp8 or w.kv_bits:
         per_tok += w.Hkv * 4 * 2  # k and v scales
     qo = w.B * w.Hq * w.D * 2 * 2 + w.B * w.Hq * 4
     return tok * per_tok + qo
@@ -302,7 +306,7 @@ def bench_decode(name, steps, warmup, world, dev, pk, paged=False, n_q=1):
         Tmax = d["page_table"].shape[1] * PAGE_SIZE
         table = d["page_table"].to(dev)
     qd, ld = d["q"].to(dev), lens.to(dev)
-    if w.kv_fp8:
+    if w.kv_fp8 or w.kv_bits:
         kd, vd = d["k_codes"].to(dev), d["v_codes"].to(dev)
         ks, vs = d["k_scale"].to(dev), d["v_scale"].to(dev)
     else:
@@ -447,8 +451,9 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=128)
     ap.add_argument("--workloads",
                     default="prefill,prefill_varlen,decode_bf16,decode_fp8,decode_bf16_paged,decode_fp8_paged,"
-                            "decode_bf16_multi,decode_fp8_multi",
-                    help="comma list of prefill, decode_bf16, decode_fp8 (profiling runs select one)")
+                            "decode_bf16_multi,decode_fp8_multi,decode_int8,decode_int4",
+                    help="comma list of prefill, prefill_varlen, decode_{bf16,fp8,int8,int4}[_paged|_multi] "
+                         "(profiling runs select one)")
     args = ap.parse_args()
     w = I.WORKLOADS[HEADLINE]
     config = {"workload": HEADLINE, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
@@ -491,7 +496,7 @@ def main():
     pre = bench_prefill(w, args.steps, args.warmup, world, dev, pk) if "prefill" in sel else None
     dec = []
     if not args.no_decode:
-        for key, name in zip(("decode_bf16", "decode_fp8"), DECODE_WORKLOADS):
+        for key, name in DECODE_WORKLOADS:
             if key in sel:
                 dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk))
             if key + "_paged" in sel:

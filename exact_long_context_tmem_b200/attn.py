@@ -21,7 +21,23 @@ ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA = 1, 2, 3
 ATTN_ERR_BUDGET, ATTN_ERR_TIMEOUT, ATTN_ERR_INJECTED = 4, 5, 6
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "budget", 5: "timeout",
           6: "injected"}
-ATTN_BF16, ATTN_FP8_E4M3, ATTN_F32 = 0, 1, 2
+ATTN_BF16, ATTN_FP8_E4M3, ATTN_F32, ATTN_INT8, ATTN_INT4 = 0, 1, 2, 3, 4
+_KV_NAMES = {"bf16": ATTN_BF16, "fp8": ATTN_FP8_E4M3, "int8": ATTN_INT8, "int4": ATTN_INT4}
+
+
+def _kv_kind(k, D: int, kv_dtype: str | None) -> int:
+    """Cache element kind: explicit ("bf16", "fp8", "int8", "int4"), else from the tensor: int8 ->
+    INT8 codes; uint8 rows of D/2 bytes -> packed INT4 codes; uint8 / float8_e4m3fn rows of D -> E4M3
+    codes; otherwise bf16."""
+    if kv_dtype is not None:
+        return _KV_NAMES[kv_dtype]
+    if k.dtype == torch.int8:
+        return ATTN_INT8
+    if k.dtype == torch.uint8 and k.shape[-1] * 2 == D:
+        return ATTN_INT4
+    if k.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return ATTN_FP8_E4M3
+    return ATTN_BF16
 
 EXPORTS = [
     "attn_prefill", "attn_decode_workspace_bytes", "attn_decode_num_splits", "attn_decode_splitkv",
@@ -164,14 +180,16 @@ def attn_decode_num_splits(B, Hq, Hkv, D, Tmax, num_splits=0, scale=1.0) -> int:
 
 
 def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: float | None = None,
-                        num_splits: int = 0, o=None, lse=None, ws=None, want_lse: bool = True, stream=None):
-    """q [B,Hq,D] bf16; k/v [B,Tmax,Hkv,D] bf16 or uint8 E4M3 codes (+ float32 scales [B,Tmax,Hkv]);
-    kv_lens int32 [B] on the device -> (o [B,Hq,D] bf16, lse [B,Hq] float32)."""
+                        num_splits: int = 0, o=None, lse=None, ws=None, want_lse: bool = True, stream=None,
+                        kv_dtype: str | None = None):
+    """q [B,Hq,D] bf16; k/v [B,Tmax,Hkv,D] bf16, uint8 E4M3 codes or int8 codes, or [B,Tmax,Hkv,D/2]
+    uint8 packed INT4 codes (+ float32 scales [B,Tmax,Hkv] for every coded cache); kv_lens int32
+    [B] on the device -> (o [B,Hq,D] bf16, lse [B,Hq] float32)."""
     _need_cuda(q, k, v, kv_lens, k_scale, v_scale)
     B, Hq, D = q.shape
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    fp8 = k.dtype in (torch.uint8, torch.float8_e4m3fn)
+    kind = _kv_kind(k, D, kv_dtype)
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -181,7 +199,7 @@ def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: 
     if ws is None and need > 0:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
-    st = lib().attn_decode_splitkv(_ptr(q), _ptr(k), _ptr(v), ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(k_scale),
+    st = lib().attn_decode_splitkv(_ptr(q), _ptr(k), _ptr(v), kind, _ptr(k_scale),
                                    _ptr(v_scale), _ptr(kv_lens), int(Tmax), dims, int(num_splits), _ptr(o),
                                    _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "attn_decode_splitkv")
@@ -211,14 +229,15 @@ def attn_prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, 
 
 
 def attn_decode_multi(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: float | None = None,
-                      num_splits: int = 0, o=None, lse=None, ws=None, want_lse: bool = True, stream=None):
+                      num_splits: int = 0, o=None, lse=None, ws=None, want_lse: bool = True, stream=None,
+                      kv_dtype: str | None = None):
     """q [B,n_q,Hq,D] bf16 (n_q new tokens per sequence, already in the cache); k/v as for
     attn_decode_splitkv -> (o [B,n_q,Hq,D] bf16, lse [B,n_q,Hq] float32)."""
     _need_cuda(q, k, v, kv_lens, k_scale, v_scale)
     B, n_q, Hq, D = q.shape
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    fp8 = k.dtype in (torch.uint8, torch.float8_e4m3fn)
+    kind = _kv_kind(k, D, kv_dtype)
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, n_q, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -228,7 +247,7 @@ def attn_decode_multi(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: fl
     if ws is None and need > 0:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
-    st = lib().attn_decode_multi(_ptr(q), _ptr(k), _ptr(v), ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(k_scale),
+    st = lib().attn_decode_multi(_ptr(q), _ptr(k), _ptr(v), kind, _ptr(k_scale),
                                  _ptr(v_scale), _ptr(kv_lens), int(Tmax), int(n_q), dims, int(num_splits), _ptr(o),
                                  _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "attn_decode_multi")
@@ -237,16 +256,17 @@ def attn_decode_multi(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: fl
 
 def attn_decode_paged(q, k_pool, v_pool, page_table, kv_lens, *, k_scale=None, v_scale=None,
                       scale: float | None = None, num_splits: int = 0, o=None, lse=None, ws=None,
-                      want_lse: bool = True, stream=None):
-    """q [B,Hq,D] bf16; k_pool/v_pool [num_pages, page_size, Hkv, D] bf16 or uint8 E4M3 codes
-    (+ float32 scale pools [num_pages, page_size, Hkv]); page_table int32 [B, max_pages] and
+                      want_lse: bool = True, stream=None, kv_dtype: str | None = None):
+    """q [B,Hq,D] bf16; k_pool/v_pool [num_pages, page_size, Hkv, D] bf16, uint8 E4M3 or int8 codes,
+    or [num_pages, page_size, Hkv, D/2] packed INT4 codes (+ float32 scale pools
+    [num_pages, page_size, Hkv] for every coded cache); page_table int32 [B, max_pages] and
     kv_lens int32 [B] on the device -> (o [B,Hq,D] bf16, lse [B,Hq] float32)."""
     _need_cuda(q, k_pool, v_pool, page_table, kv_lens, k_scale, v_scale)
     B, Hq, D = q.shape
     num_pages, page_size, Hkv = k_pool.shape[0], k_pool.shape[1], k_pool.shape[2]
     max_pages = page_table.shape[1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    fp8 = k_pool.dtype in (torch.uint8, torch.float8_e4m3fn)
+    kind = _kv_kind(k_pool, D, kv_dtype)
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -256,7 +276,7 @@ def attn_decode_paged(q, k_pool, v_pool, page_table, kv_lens, *, k_scale=None, v
     if ws is None and need > 0:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
-    st = lib().attn_decode_paged(_ptr(q), _ptr(k_pool), _ptr(v_pool), ATTN_FP8_E4M3 if fp8 else ATTN_BF16,
+    st = lib().attn_decode_paged(_ptr(q), _ptr(k_pool), _ptr(v_pool), kind,
                                  _ptr(k_scale), _ptr(v_scale), _ptr(page_table), int(max_pages), int(page_size),
                                  int(num_pages), _ptr(kv_lens), dims, int(num_splits), _ptr(o), _ptr(lse), _ptr(ws),
                                  ws_bytes, _stream(stream))
@@ -268,7 +288,8 @@ NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 def attn_decode_splitkv_noalloc(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: float | None = None,
-                                num_splits: int = 0, o=None, lse=None, want_lse: bool = True, stream=None):
+                                num_splits: int = 0, o=None, lse=None, want_lse: bool = True, stream=None,
+                                kv_dtype: str | None = None):
     """attn_decode_splitkv without a workspace: the split partials live in the library's static
     device scratch array (see include/attn.h).  For callers that cannot allocate device memory;
     the outputs o and lse may be passed in preallocated."""
@@ -276,12 +297,12 @@ def attn_decode_splitkv_noalloc(q, k, v, kv_lens, *, k_scale=None, v_scale=None,
     B, Hq, D = q.shape
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    fp8 = k.dtype in (torch.uint8, torch.float8_e4m3fn)
+    kind = _kv_kind(k, D, kv_dtype)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    st = lib().attn_decode_splitkv_noalloc(_ptr(q), _ptr(k), _ptr(v), ATTN_FP8_E4M3 if fp8 else ATTN_BF16,
+    st = lib().attn_decode_splitkv_noalloc(_ptr(q), _ptr(k), _ptr(v), kind,
                                            _ptr(k_scale), _ptr(v_scale), _ptr(kv_lens), int(Tmax),
                                            _dims(B, Hq, Hkv, D, scale), int(num_splits), _ptr(o), _ptr(lse),
                                            _stream(stream))

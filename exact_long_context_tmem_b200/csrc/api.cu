@@ -14,6 +14,7 @@
 #include "../../include/attn.h"
 #include "decode.cuh"
 #include "decode_fp8.cuh"
+#include "decode_int.cuh"
 #include "merge.cuh"
 #include "prefill.cuh"
 
@@ -54,9 +55,11 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 4-D tiled map over a row-major [d3][d2][d1][d0] tensor, 128-byte swizzle, zero fill out of bounds.
+// 4-D tiled map over a row-major [d3][d2][d1][d0] tensor, 128-byte swizzle (or `swz`), zero fill out
+// of bounds.
 static attn_status_t make_map_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes,
-                                 const uint64_t dims[4], const uint32_t box[4]) {
+                                 const uint64_t dims[4], const uint32_t box[4],
+                                 CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t gdim[4] = {dims[0], dims[1], dims[2], dims[3]};
@@ -64,8 +67,8 @@ static attn_status_t make_map_4d(CUtensorMap* map, const void* base, CUtensorMap
                            dims[0] * dims[1] * dims[2] * elem_bytes};
   cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     t_last_cuda_error = (int)r;
     return ATTN_ERR_CUDA;
@@ -218,18 +221,49 @@ struct DecodePaging {
   int max_pages, page_size, num_pages;
 };
 
-template <bool FP8>
+template <int GP, int BITS>
+static attn_status_t launch_decode_int_gp(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p,
+                                          dim3 grid, cudaStream_t stream) {
+  static std::atomic<uint64_t> smem_done{0};
+  attn_status_t st = ensure_smem(decode_int_sm100<GP, BITS>, DecodeIntCfg<BITS>::SMEM_BYTES, smem_done);
+  if (st != ATTN_OK) return st;
+  decode_int_sm100<GP, BITS><<<grid, DecodeIntCfg<BITS>::THREADS, DecodeIntCfg<BITS>::SMEM_BYTES, stream>>>(mk, mv, p);
+  ATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+template <int BITS>
+static attn_status_t launch_decode_int(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int R,
+                                       dim3 grid, cudaStream_t stream) {
+  if (R <= 1) return launch_decode_int_gp<1, BITS>(mk, mv, p, grid, stream);
+  if (R <= 2) return launch_decode_int_gp<2, BITS>(mk, mv, p, grid, stream);
+  if (R <= 4) return launch_decode_int_gp<4, BITS>(mk, mv, p, grid, stream);
+  if (R <= 8) return launch_decode_int_gp<8, BITS>(mk, mv, p, grid, stream);
+  return launch_decode_int_gp<16, BITS>(mk, mv, p, grid, stream);
+}
+
+// Cache element kinds of the decode launcher.
+enum DecodeKv { KV_BF16 = 0, KV_FP8 = 1, KV_INT8 = 2, KV_INT4 = 3 };
+
+template <int KV>
 static attn_status_t launch_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
                                    const int* kv_lens, int Tmax, const attn_dims_t& d, int P, int split_tokens,
                                    void* o, float* lse, void* ws, cudaStream_t stream, const DecodePaging& pg,
                                    int n_q = 1) {
+  constexpr bool FP8 = KV == KV_FP8;
   attn_status_t st;
   CUtensorMap mk, mv;
   // With Tmax == 0 every split is empty and no map is read; it still needs a valid base and extent.
-  const uint64_t dk[4] = {128, (uint64_t)d.Hkv, (uint64_t)std::max(pg.page_size, 1), (uint64_t)std::max(pg.num_pages, 1)};
+  const uint64_t row = KV == KV_INT4 ? 64 : 128;  // elements (bytes for the 8-bit and 4-bit caches) per row
+  const uint64_t dk[4] = {row, (uint64_t)d.Hkv, (uint64_t)std::max(pg.page_size, 1), (uint64_t)std::max(pg.num_pages, 1)};
   const void* kb = Tmax > 0 ? k : q;
   const void* vb = Tmax > 0 ? v : q;
-  if (FP8) {
+  if (KV == KV_INT8 || KV == KV_INT4) {
+    const uint32_t box[4] = {(uint32_t)row, 1, 128, 1};
+    const CUtensorMapSwizzle swz = KV == KV_INT4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    if ((st = make_map_4d(&mk, kb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dk, box, swz)) != ATTN_OK) return st;
+    if ((st = make_map_4d(&mv, vb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dk, box, swz)) != ATTN_OK) return st;
+  } else if (FP8) {
     const uint32_t box[4] = {128, 1, 128, 1};
     if ((st = make_map_4d(&mk, kb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dk, box)) != ATTN_OK) return st;
     if ((st = make_map_4d(&mv, vb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dk, box)) != ATTN_OK) return st;
@@ -268,7 +302,10 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
   // The query group is padded to the next power of two (<= 16) so the kernels' per-row loops unroll.
   const int R = p.G * n_q;  // MMA rows of one (sequence, KV head)
   // Single-token decode runs instances without per-row key limits (one compare per token).
-  if (n_q == 1) {
+  if (KV == KV_INT8 || KV == KV_INT4) {
+    if (n_q != 1) return ATTN_ERR_UNSUPPORTED;
+    st = launch_decode_int<KV == KV_INT8 ? 8 : 4>(mk, mv, p, R, grid, stream);
+  } else if (n_q == 1) {
     if (R <= 1) st = launch_decode_gp<FP8, 1, false>(mk, mv, p, grid, stream);
     else if (R <= 2) st = launch_decode_gp<FP8, 2, false>(mk, mv, p, grid, stream);
     else if (R <= 4) st = launch_decode_gp<FP8, 4, false>(mk, mv, p, grid, stream);
@@ -296,6 +333,23 @@ static attn_status_t launch_decode(const void* q, const void* k, const void* v, 
     ATTN_CUDA(cudaGetLastError());
   }
   return ATTN_OK;
+}
+
+static bool kv_dtype_ok(attn_dtype_t t) {
+  return t == ATTN_BF16 || t == ATTN_FP8_E4M3 || t == ATTN_INT8 || t == ATTN_INT4;
+}
+
+// Single-token decode over a cache of any supported element kind.
+static attn_status_t launch_decode_kind(attn_dtype_t kv, const void* q, const void* k, const void* v, const float* ks,
+                                        const float* vs, const int* kv_lens, int Tmax, const attn_dims_t& d, int P,
+                                        int per, void* o, float* lse, void* ws, cudaStream_t st,
+                                        const DecodePaging& pg) {
+  switch (kv) {
+    case ATTN_FP8_E4M3: return launch_decode<KV_FP8>(q, k, v, ks, vs, kv_lens, Tmax, d, P, per, o, lse, ws, st, pg);
+    case ATTN_INT8: return launch_decode<KV_INT8>(q, k, v, ks, vs, kv_lens, Tmax, d, P, per, o, lse, ws, st, pg);
+    case ATTN_INT4: return launch_decode<KV_INT4>(q, k, v, ks, vs, kv_lens, Tmax, d, P, per, o, lse, ws, st, pg);
+    default: return launch_decode<KV_BF16>(q, k, v, nullptr, nullptr, kv_lens, Tmax, d, P, per, o, lse, ws, st, pg);
+  }
 }
 
 // ---------------------------------------------------------------- diagnostics
@@ -431,14 +485,14 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, a
                                   attn_dims_t dims, int num_splits, void* o, float* lse, void* ws, size_t ws_bytes,
                                   void* stream) {
   if (!dims_ok(dims) || Tmax < 0 || num_splits < 0 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
-  if (kv_dtype != ATTN_BF16 && kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (!kv_dtype_ok(kv_dtype)) return ATTN_ERR_INVALID_ARG;
   if (dims.B == 0) return ATTN_OK;
   if (!q || !o || !kv_lens || (Tmax > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
-  const bool fp8 = kv_dtype == ATTN_FP8_E4M3;
-  if (fp8 != (k_scale != nullptr) || fp8 != (v_scale != nullptr)) return ATTN_ERR_INVALID_ARG;
+  const bool quant = kv_dtype != ATTN_BF16;  // codes + per-token scales
+  if (quant != (k_scale != nullptr) || quant != (v_scale != nullptr)) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned4(kv_lens) || (lse && !aligned4(lse))) return ATTN_ERR_INVALID_ARG;
   if (Tmax > 0 && (!aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
-  if (fp8 && (!aligned4(k_scale) || !aligned4(v_scale))) return ATTN_ERR_INVALID_ARG;
+  if (quant && (!aligned4(k_scale) || !aligned4(v_scale))) return ATTN_ERR_INVALID_ARG;
   if (dims.D != 128 || dims.Hq / dims.Hkv > 16) return ATTN_ERR_UNSUPPORTED;
   if (dims.B > 65535 || dims.Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
   const int P = decode_splits(dims, Tmax, num_splits);
@@ -447,8 +501,7 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, a
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int per = decode_split_tokens(Tmax, P);
   const DecodePaging pg{nullptr, 1, Tmax, dims.B};
-  if (fp8) return launch_decode<true>(q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
-  return launch_decode<false>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
+  return launch_decode_kind(kv_dtype, q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
 }
 
 attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, attn_dtype_t kv_dtype,
@@ -456,18 +509,18 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v
                                 int max_pages, int page_size, int num_pages, const int* kv_lens, attn_dims_t dims,
                                 int num_splits, void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (!dims_ok(dims) || num_splits < 0 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
-  if (kv_dtype != ATTN_BF16 && kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (!kv_dtype_ok(kv_dtype)) return ATTN_ERR_INVALID_ARG;
   if (max_pages < 1 || page_size < 128 || page_size % 128 != 0 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
   if ((long long)max_pages * page_size > 0x7fffffffLL || (long long)num_pages * page_size > 0x7fffffffLL)
     return ATTN_ERR_UNSUPPORTED;
   if (dims.B == 0) return ATTN_OK;
   if (!q || !o || !kv_lens || !page_table || !k_pool || !v_pool) return ATTN_ERR_INVALID_ARG;
-  const bool fp8 = kv_dtype == ATTN_FP8_E4M3;
-  if (fp8 != (k_scale_pool != nullptr) || fp8 != (v_scale_pool != nullptr)) return ATTN_ERR_INVALID_ARG;
+  const bool quant = kv_dtype != ATTN_BF16;  // codes + per-token scales
+  if (quant != (k_scale_pool != nullptr) || quant != (v_scale_pool != nullptr)) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned4(kv_lens) || !aligned4(page_table) || (lse && !aligned4(lse)))
     return ATTN_ERR_INVALID_ARG;
   if (!aligned16(k_pool) || !aligned16(v_pool)) return ATTN_ERR_INVALID_ARG;
-  if (fp8 && (!aligned4(k_scale_pool) || !aligned4(v_scale_pool))) return ATTN_ERR_INVALID_ARG;
+  if (quant && (!aligned4(k_scale_pool) || !aligned4(v_scale_pool))) return ATTN_ERR_INVALID_ARG;
   if (dims.D != 128 || dims.Hq / dims.Hkv > 16) return ATTN_ERR_UNSUPPORTED;
   if (dims.B > 65535 || dims.Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
   const int Tmax = max_pages * page_size;
@@ -477,10 +530,8 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int per = decode_split_tokens(Tmax, P);
   const DecodePaging pg{page_table, max_pages, page_size, num_pages};
-  if (fp8)
-    return launch_decode<true>(q, k_pool, v_pool, k_scale_pool, v_scale_pool, kv_lens, Tmax, dims, P, per, o, lse, ws,
-                               st, pg);
-  return launch_decode<false>(q, k_pool, v_pool, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg);
+  return launch_decode_kind(kv_dtype, q, k_pool, v_pool, k_scale_pool, v_scale_pool, kv_lens, Tmax, dims, P, per, o,
+                            lse, ws, st, pg);
 }
 
 size_t attn_decode_multi_workspace_bytes(attn_dims_t dims, int Tmax, int n_q, int num_splits) {
@@ -493,7 +544,8 @@ attn_status_t attn_decode_multi(const void* q, const void* k, const void* v, att
                                 attn_dims_t dims, int num_splits, void* o, float* lse, void* ws, size_t ws_bytes,
                                 void* stream) {
   if (!dims_ok(dims) || Tmax < 0 || num_splits < 0 || num_splits > 4096 || n_q < 1) return ATTN_ERR_INVALID_ARG;
-  if (kv_dtype != ATTN_BF16 && kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (!kv_dtype_ok(kv_dtype)) return ATTN_ERR_INVALID_ARG;
+  if (kv_dtype == ATTN_INT8 || kv_dtype == ATTN_INT4) return ATTN_ERR_UNSUPPORTED;
   if (dims.B == 0) return ATTN_OK;
   if (!q || !o || !kv_lens || (Tmax > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
   const bool fp8 = kv_dtype == ATTN_FP8_E4M3;
@@ -509,8 +561,8 @@ attn_status_t attn_decode_multi(const void* q, const void* k, const void* v, att
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int per = decode_split_tokens(Tmax, P);
   const DecodePaging pg{nullptr, 1, Tmax, dims.B};
-  if (fp8) return launch_decode<true>(q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg, n_q);
-  return launch_decode<false>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg, n_q);
+  if (fp8) return launch_decode<KV_FP8>(q, k, v, k_scale, v_scale, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg, n_q);
+  return launch_decode<KV_BF16>(q, k, v, nullptr, nullptr, kv_lens, Tmax, dims, P, per, o, lse, ws, st, pg, n_q);
 }
 
 // Split-KV decode without allocation: the split partials live in this static device array

@@ -1,0 +1,516 @@
+// Split-KV GQA decode over an INT8 or INT4 KV cache (ORT CPU GQA analysis: the KV cache is held
+// as INT8 / INT4 codes and V is dequantised on the fly inside the SV accumulation; "Flash
+// Decoding": the key range is split and the partial softmax states are merged by log-sum-exp).
+//
+// Codes: INT8 is one two's complement byte per element; INT4 is two 4-bit two's complement
+// elements per byte, element 2i in the low nibble of byte i (a 128-element row is 64 bytes).  Each
+// (token, KV head) has one float32 scale for K and one for V; value = code * scale.
+//
+// The dequantisation is fused into the tile load.  TMA brings the raw code tiles into shared
+// memory; converter warps widen them to f16 (exact: every INT8 and INT4 value is an f16 value) -- K
+// straight into TMEM as the A operand of S^T = K . Q^T, V into shared memory as the A operand of
+// O^T += V^T . P^T -- and the scales stay out of the operands: k_scale multiplies the token's score
+// and v_scale its probability, on the thread that owns the token.
+//
+// Q is one f16 row per query head, scaled by a power of two 2^e that puts the row's absmax in
+// [2^14, 2^15): every bf16 element within 2^31 of the row max is then an exact f16, and the score
+// is S_mma * 2^-e.  The running max is taken over y = x + log2(v_scale) (x the log2-domain score),
+// so the probability that enters P, 2^(y - m) = 2^(x - m) * v_scale, stays below 2^threshold
+// whatever the scale; the row sum l adds 2^(x - m) = P / v_scale.
+//
+// Roles (480 threads, one CTA per (split, KV head, sequence)):
+//   warp 0       TMA producer of the raw K code tiles (NCS-stage ring)
+//   warp 14      TMA producer of the raw V code tiles (NCS-stage ring)
+//   warp 1       TMEM allocator; lane 0 issues every MMA
+//   warps 2..5   K converter: thread = token; codes -> f16 into TMEM
+//   warps 6..9   V converter: thread = token; codes -> f16 in shared memory (MN-major operand)
+//   warps 10..13 Q staging, softmax, epilogue: thread = token (later = output element d)
+// Scores, probabilities and converted tiles rotate through NB = 3 buffers: S(j+3) is issued right
+// after PV(j).  TMEM columns: S^T [0, 48) (three 16-column buffers), O^T [48, 64), converted K
+// [64, 256) (three 64-column buffers, 128 f16 per lane).
+#pragma once
+
+#include "decode.cuh"
+
+namespace attn {
+
+template <int BITS>
+struct DecodeIntCfg {
+  static constexpr int D = 128;
+  static constexpr int ROW = BITS == 8 ? 128 : 64;  // code bytes per token row
+  static constexpr int NCS = 3;                     // stages of raw code tiles
+  static constexpr int NB = 3;                      // S / P / converted-tile buffers
+  static constexpr int CODE_TILE = 128 * ROW;
+  static constexpr int VC_TILE = 2 * 128 * 128;     // 128 tokens x 128 f16, two 64-wide boxes
+  static constexpr int QBOX = 16 * 128;             // 16 rows x 64 f16
+  static constexpr int Q_BYTES = 2 * QBOX;
+  static constexpr int PBOX = 16 * 128;
+  static constexpr int P_BYTES = 2 * PBOX;
+  static constexpr int OFF_KCODE = 0;
+  static constexpr int OFF_VCODE = OFF_KCODE + NCS * CODE_TILE;
+  static constexpr int OFF_VC = OFF_VCODE + NCS * CODE_TILE;
+  static constexpr int OFF_Q = OFF_VC + NB * VC_TILE;
+  static constexpr int OFF_P = OFF_Q + Q_BYTES;
+  static constexpr int OFF_RED = OFF_P + NB * P_BYTES;
+  static constexpr int OFF_QSC = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;  // [16] 2^-e per query row
+  static constexpr int OFF_BAR = OFF_QSC + 16 * 4;
+  static constexpr int N_BARS = 4 * NCS + 1 + 7 * NB + 1 + 2 + 1 + 1;
+  static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
+  static constexpr int THREADS = 480;
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t COL_S = 0, COL_O = 48, COL_K = 64;
+  static constexpr float RESCALE_THRESHOLD = 8.0f;
+};
+static_assert(DecodeIntCfg<8>::SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+static_assert(DecodeIntCfg<4>::SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+static_assert(DecodeIntCfg<8>::OFF_VCODE % 1024 == 0 && DecodeIntCfg<4>::OFF_VCODE % 1024 == 0, "TMA tile alignment");
+
+// Byte offset of 16-byte chunk c of token row t in a TMA code tile: 128-byte rows with the 128B
+// swizzle (INT8), 64-byte rows with the 64B swizzle (INT4: chunk c ^ bits 7..8 of the address).
+template <int BITS>
+__device__ __forceinline__ uint32_t int_code_offset(uint32_t t, uint32_t c) {
+  if (BITS == 8) return sw128_offset(t, c);
+  return t * 64u + ((c ^ ((t >> 1) & 3u)) << 4);
+}
+
+__device__ __forceinline__ uint32_t sub_f16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Four INT8 codes -> f16 pairs (elements 0,1) and (2,3), exact: code + 128 becomes the low 8
+// mantissa bits of an f16 in [1024, 2048), whose unit in the last place is 1; 1152 is subtracted.
+__device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t& h01, uint32_t& h23) {
+  const uint32_t u = w ^ 0x80808080u;
+  h01 = sub_f16x2(__byte_perm(u, 0x64646464u, 0x5150u), 0x64806480u);
+  h23 = sub_f16x2(__byte_perm(u, 0x64646464u, 0x5352u), 0x64806480u);
+}
+
+// Eight INT4 codes (one word; element k in nibble k) -> four f16 pairs in element order, exact:
+// code + 8 becomes the low 4 mantissa bits of an f16 in [1024, 1040); 1032 is subtracted.
+__device__ __forceinline__ void i4x8_to_f16(uint32_t w, uint32_t* h) {
+  const uint32_t u = w ^ 0x88888888u;
+  const uint32_t a = (u & 0x000F000Fu) | 0x64006400u;          // elements 0, 4
+  const uint32_t b = ((u >> 4) & 0x000F000Fu) | 0x64006400u;   // 1, 5
+  const uint32_t c = ((u >> 8) & 0x000F000Fu) | 0x64006400u;   // 2, 6
+  const uint32_t d = ((u >> 12) & 0x000F000Fu) | 0x64006400u;  // 3, 7
+  h[0] = sub_f16x2(__byte_perm(a, b, 0x5410u), 0x64086408u);
+  h[1] = sub_f16x2(__byte_perm(c, d, 0x5410u), 0x64086408u);
+  h[2] = sub_f16x2(__byte_perm(a, b, 0x7632u), 0x64086408u);
+  h[3] = sub_f16x2(__byte_perm(c, d, 0x7632u), 0x64086408u);
+}
+
+// Elements [64 half, 64 half + 64) of token row t of a code tile as 32 f16 pairs (zeros when the
+// token is not valid).
+template <int BITS>
+__device__ __forceinline__ void int_row_half_to_f16(const uint8_t* tile, int t, int half, bool valid,
+                                                    uint32_t (&h)[32]) {
+  constexpr int CH = BITS == 8 ? 4 : 2;  // 16-byte code chunks per 64 elements
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (valid) w = *reinterpret_cast<const uint4*>(tile + int_code_offset<BITS>(t, half * CH + k));
+    const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (BITS == 8) i8x4_to_f16(wd[i], h[k * 8 + 2 * i], h[k * 8 + 2 * i + 1]);
+      else i4x8_to_f16(wd[i], &h[k * 16 + 4 * i]);
+    }
+  }
+}
+
+// Index of the (token, KV head) scale of sequence b's token tok, or -1 for an unmapped page.
+__device__ __forceinline__ long long int_scale_index(const DecodeParams& p, int b, int tok, int kvh) {
+  long long page = b;
+  int off = tok;
+  if (p.page_table) {
+    const int raw = __ldg(p.page_table + (long long)b * p.max_pages + tok / p.page_size);
+    if (raw < 0 || raw >= p.num_pages) return -1;
+    page = raw;
+    off = tok % p.page_size;
+  }
+  return (page * p.page_size + off) * p.Hkv + kvh;
+}
+
+// Query rows of the group as f16 rows scaled by 2^e (absmax in [2^14, 2^15); e clamped to
+// [-100, 100]) into the 128B-swizzled K-major B operand (two 64-wide boxes of 16 rows); 2^-e of
+// row g goes to qsc[g].  128 threads: chunk c = tid + 128 k is row c / 16, elements 8 (c % 16)..,
+// so the 16 threads of a row are 16 consecutive lanes of one warp.
+__device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kvh, int b, int tid, uint8_t* q_smem,
+                                            float* qsc) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int c = tid + 128 * k;
+    const int g = c >> 4, cc = c & 15;
+    const uint4 x = decode_q_chunk_load(p, G, kvh, b, c);
+    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+    float f[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(xw[i] << 16);
+      f[2 * i + 1] = __uint_as_float(xw[i] & 0xFFFF0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int e = 14 - ((int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127);
+    e = e < -100 ? -100 : (e > 100 ? 100 : e);
+    const float up = __uint_as_float((uint32_t)(e + 127) << 23);
+    uint32_t hv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hv[i] = pack_f16x2(f[2 * i] * up, f[2 * i + 1] * up);
+    *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * (16 * 128) + sw128_offset(g, cc & 7)) =
+        make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    if (cc == 0) qsc[g] = __uint_as_float((uint32_t)(127 - e) << 23);
+  }
+}
+
+// One tile of the softmax on the thread that owns token t, with the running max over
+// y = x + log2(v_scale): row maxima (warp redux, then the cross-warp exchange) -> lazy O rescale
+// -> this token's entries of P^T (2^(y - m), f16).  Returns false, warp-uniformly, if a bounded
+// wait ran out.  The parities follow decode_softmax_core.
+template <int GP>
+__device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, int lane, int wq, int t, bool valid,
+                                                 const float (&scq)[GP], float ks, float vs, uint32_t tS_lane,
+                                                 uint32_t tO_lane, float* red_max, uint64_t* red_bar,
+                                                 uint64_t* prev_pv, uint32_t prev_pv_parity, uint8_t* p_tile,
+                                                 float threshold) {
+  uint32_t sv[16];
+  tmem_ld16(tS_lane, sv);
+  tmem_wait_ld();
+  const float avs = fminf(fmaxf(fabsf(vs), 0x1p-100f), 0x1p100f);
+  const float lvs = __log2f(avs);
+  const float ivs = __frcp_rn(avs);
+  const bool neg = vs < 0.f;
+  float y[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) y[g] = valid ? fmaf(__uint_as_float(sv[g]) * scq[g], ks, lvs) : -INFINITY;
+  float* rm = red_max + (j & 1) * 64;
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float m = warp_max_redux(y[g]);
+    if (lane == 0) rm[wq * 16 + g] = m;
+  }
+  mbar_arrive(&red_bar[j & 1]);
+  if (!mbar_wait_warp(&red_bar[j & 1], (j >> 1) & 1, SITE_DC_SM_S)) return false;
+  bool need = false;
+  float alpha[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float tm = fmaxf(fmaxf(rm[g], rm[16 + g]), fmaxf(rm[32 + g], rm[48 + g]));
+    const float mn = fmaxf(rows.m_used[g], tm);
+    alpha[g] = 1.f;
+    if (mn > rows.m_used[g] + threshold) {  // the same decision on every thread of the CTA
+      alpha[g] = ex2_approx(rows.m_used[g] - mn);
+      rows.m_used[g] = mn;
+      rows.l_part[g] *= alpha[g];
+      need = true;
+    }
+  }
+  if (need && j > 0) {  // rescale O^T row t once the previous PV is done
+    if (!mbar_wait_warp(prev_pv, prev_pv_parity, SITE_DC_SM_O)) return false;
+    tc_fence_after();
+    uint32_t orow[16];
+    tmem_ld16(tO_lane, orow);
+    tmem_wait_ld();
+#pragma unroll
+    for (int g = 0; g < GP; ++g) orow[g] = __float_as_uint(__uint_as_float(orow[g]) * alpha[g]);
+    tmem_st16(tO_lane, orow);
+    tmem_wait_st();
+  }
+  uint8_t* prow = p_tile + (t >> 6) * (16 * 128);
+  const uint32_t pchunk = (t & 63) >> 3, pbyte = (t & 7) * 2;
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float pe = (y[g] == -INFINITY) ? 0.f : ex2_approx(y[g] - rows.m_used[g]);
+    rows.l_part[g] += pe * ivs;
+    *reinterpret_cast<uint16_t*>(prow + sw128_offset(g, pchunk) + pbyte) =
+        __half_as_ushort(__float2half_rn(neg ? -pe : pe));
+  }
+  return true;
+}
+
+template <int GP, int BITS>
+__global__ void __launch_bounds__(480, 1)
+    decode_int_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const DecodeParams p) {
+  using C = DecodeIntCfg<BITS>;
+  constexpr int NB = C::NB;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int len = p.kv_lens[b];
+  len = len < 0 ? 0 : (len > p.Tmax ? p.Tmax : len);
+  const int t0 = split * p.split_tokens;
+  const int t1 = min(len, t0 + p.split_tokens);
+  const int n = t1 > t0 ? (t1 - t0 + 127) / 128 : 0;
+  const int G = p.G;
+
+  if (n == 0) {
+    decode_write_empty(p, G, split, kvh, b, threadIdx.x, blockDim.x);
+    return;
+  }
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* k_full = bars;              // [NCS] raw K codes landed
+  uint64_t* k_empty = k_full + C::NCS;  // [NCS] converter done with the raw K stage
+  uint64_t* v_full = k_empty + C::NCS;
+  uint64_t* v_empty = v_full + C::NCS;
+  uint64_t* q_ready = v_empty + C::NCS;
+  uint64_t* s_full = q_ready + 1;    // [NB] S^T(j) in TMEM
+  uint64_t* p_full = s_full + NB;    // [NB] P^T(j) in shared memory
+  uint64_t* pv_done = p_full + NB;   // [NB] PV(j) completed
+  uint64_t* kc_full = pv_done + NB;  // [NB] converted K in TMEM
+  uint64_t* kc_empty = kc_full + NB; // [NB] S MMA done reading it
+  uint64_t* vc_full = kc_empty + NB; // [NB] converted V in shared memory
+  uint64_t* vc_empty = vc_full + NB; // [NB] PV MMA done reading it
+  uint64_t* drain = vc_empty + NB;
+  uint64_t* red_bar = drain + 1;  // [2]
+  uint64_t* sum_bar = red_bar + 2;
+  uint64_t* o_final = sum_bar + 1;  // single phase: every PV of the split has completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_final + 1);
+  float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][16]
+  float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
+  float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NCS; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 128);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 128);
+    }
+    mbar_init(q_ready, 128);
+    for (int s = 0; s < NB; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&pv_done[s], 1);
+      mbar_init(&kc_full[s], 128);
+      mbar_init(&kc_empty[s], 1);
+      mbar_init(&vc_full[s], 128);
+      mbar_init(&vc_empty[s], 1);
+    }
+    mbar_init(&red_bar[0], 128);
+    mbar_init(&red_bar[1], 128);
+    mbar_init(drain, 1);
+    mbar_init(sum_bar, 128);
+    mbar_init(o_final, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tS0 = tmem + C::COL_S, tO = tmem + C::COL_O, tK0 = tmem + C::COL_K;
+
+  if (warp == 0 || warp == 14) {
+    // ------------------------------------------------------------------ TMA producers (K: warp 0, V: warp 14)
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      const CUtensorMap* tm = is_k ? &tmK : &tmV;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      uint8_t* ring = smem + (is_k ? C::OFF_KCODE : C::OFF_VCODE);
+      tma_prefetch_desc(tm);
+      PageCursor pc;
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % C::NCS;
+        if (!(ok = mbar_wait(&empty[st], ((j / C::NCS) & 1) ^ 1, SITE_DC_LOAD_EMPTY))) break;
+        const int tok = t0 + j * 128;
+        const int page = pc.get(p, b, tok);
+        mbar_arrive_expect_tx(&full[st], C::CODE_TILE);
+        tma_load_4d(ring + st * C::CODE_TILE, tm, &full[st], 0, kvh, pc.offset(p, tok), page);
+        issued = j + 1;
+      }
+      if (!ok)  // wait (bounded) for the copies still in flight before the CTA exits
+        for (int j = (issued > C::NCS ? issued - C::NCS : 0); j < issued; ++j)
+          mbar_wait_drain(&full[j % C::NCS], (j / C::NCS) & 1, SITE_DC_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc_f16(128, 16, false, false, false);
+      constexpr uint32_t idesc_pv = make_idesc_f16(128, 16, true, false, false);
+      const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+      const uint32_t sP = smem_u32(smem + C::OFF_P);
+      const uint32_t sVc = smem_u32(smem + C::OFF_VC);
+      // S^T(j) [128 x 16] = K_j (TMEM, f16) . Q^T
+      auto issue_s = [&](int buf) {
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t qoff = (kk >> 2) * C::QBOX + (kk & 3) * 32;
+          mma_ts(tS0 + buf * 16, tK0 + buf * 64 + kk * 8, make_sdesc_sw128(sQ + qoff, 16, 1024), idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int buf, bool acc) {  // O^T += V_j^T . P_j^T
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = make_sdesc_sw128(sVc + buf * C::VC_TILE + kk * 16 * 128, 128 * 128, 1024);
+          const uint64_t db = make_sdesc_sw128(sP + buf * C::P_BYTES + (kk >> 2) * C::PBOX + (kk & 3) * 32, 16, 1024);
+          mma_ss(tO, da, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_ready, 0, SITE_DC_MMA_K);
+      for (int jj = 0; jj < NB && jj < n && ok; ++jj) {
+        if (!(ok = mbar_wait(&kc_full[jj], 0, SITE_DC_MMA_K))) break;
+        tc_fence_after();
+        issue_s(jj);
+        mma_commit(&s_full[jj]);
+        mma_commit(&kc_empty[jj]);
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int bj = j % NB;
+        const uint32_t ph = (j / NB) & 1;
+        if (!(ok = mbar_wait(&vc_full[bj], ph, SITE_DC_MMA_V))) break;
+        if (!(ok = mbar_wait(&p_full[bj], ph, SITE_DC_MMA_P))) break;
+        tc_fence_after();
+        issue_pv(bj, j > 0);
+        mma_commit(&pv_done[bj]);
+        mma_commit(&vc_empty[bj]);
+        if (j + NB < n) {  // S(j+NB) reuses buffer bj: S(j) was read before P(j) was published
+          if (!(ok = mbar_wait(&kc_full[bj], ph ^ 1, SITE_DC_MMA_K))) break;
+          tc_fence_after();
+          issue_s(bj);
+          mma_commit(&s_full[bj]);
+          mma_commit(&kc_empty[bj]);
+        }
+      }
+      if (ok) mma_commit(o_final);
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, SITE_DC_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ K converter warpgroup
+    const int wq = warp & 3;
+    const int t = wq * 32 + lane;  // token row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % C::NCS;
+      const uint32_t ph = (j / C::NCS) & 1;
+      const int bj = j % NB;
+      const uint32_t phb = (j / NB) & 1;
+      const bool valid = t0 + j * 128 + t < t1;
+      if (!mbar_wait_warp(&k_full[st], ph, SITE_DC_SM_K)) break;
+      if (!mbar_wait_warp(&kc_empty[bj], phb ^ 1, SITE_DC_SM_K)) break;  // S(j-NB) has read it
+      tc_fence_after();
+      const uint8_t* ktile = smem + C::OFF_KCODE + st * C::CODE_TILE;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t h[32];
+        int_row_half_to_f16<BITS>(ktile, t, half, valid, h);
+        tmem_st32(tK0 + bj * 64 + half * 32 + lane_off, h);
+      }
+      tmem_wait_st();
+      mbar_arrive(&k_empty[st]);
+      tc_fence_before();
+      mbar_arrive(&kc_full[bj]);
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------------ V converter warpgroup
+    const int t = (warp & 3) * 32 + lane;  // token row of the tile
+    for (int j = 0; j < n; ++j) {
+      const int st = j % C::NCS;
+      const uint32_t ph = (j / C::NCS) & 1;
+      const int bj = j % NB;
+      const uint32_t phb = (j / NB) & 1;
+      const bool valid = t0 + j * 128 + t < t1;
+      if (!mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V)) break;
+      if (!mbar_wait_warp(&vc_empty[bj], phb ^ 1, SITE_DC_SM_V)) break;  // PV(j-NB) has read it
+      const uint8_t* vtile = smem + C::OFF_VCODE + st * C::CODE_TILE;
+      uint8_t* vc = smem + C::OFF_VC + bj * C::VC_TILE;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // elements [64 half, +64) = box `half` of the operand
+        uint32_t h[32];
+        int_row_half_to_f16<BITS>(vtile, t, half, valid, h);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(vc + half * (128 * 128) + sw128_offset(t, k)) =
+              make_uint4(h[4 * k], h[4 * k + 1], h[4 * k + 2], h[4 * k + 3]);
+      }
+      mbar_arrive(&v_empty[st]);
+      fence_proxy_async_smem();
+      mbar_arrive(&vc_full[bj]);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroup
+    const int wq = warp & 3;
+    const int t = wq * 32 + lane;  // token of the tile / TMEM lane / output element d
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int wg_tid = threadIdx.x - 320;
+    for (int i = wg_tid; i < NB * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
+      reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
+    int_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, qsc);
+    fence_proxy_async_smem();
+    mbar_arrive(q_ready);
+    named_barrier_sync(1, 128);  // every row's 2^-e is in qsc
+    float scq[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) scq[g] = p.scale_log2 * qsc[g];
+
+    DecodeRows<GP> rows;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      rows.m_used[g] = -INFINITY;
+      rows.l_part[g] = 0.f;
+    }
+    bool ok = true;
+    // Per-token scales are prefetched one tile ahead so their global-memory latency stays off
+    // the tile's critical path; an unmapped page leaves them at 1 (its codes land as zeros).
+    float ks_next = 1.f, vs_next = 1.f;
+    if (t0 + t < t1) {
+      const long long i = int_scale_index(p, b, t0 + t, kvh);
+      if (i >= 0) {
+        ks_next = __ldg(p.k_scale + i);
+        vs_next = __ldg(p.v_scale + i);
+      }
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const int bj = j % NB;
+      const uint32_t phb = (j / NB) & 1;
+      const int tok = t0 + j * 128 + t;
+      const bool valid = tok < t1;
+      const float ks = ks_next, vs = vs_next;
+      ks_next = 1.f;
+      vs_next = 1.f;
+      if (tok + 128 < t1) {
+        const long long i = int_scale_index(p, b, tok + 128, kvh);
+        if (i >= 0) {
+          ks_next = __ldg(p.k_scale + i);
+          vs_next = __ldg(p.v_scale + i);
+        }
+      }
+      if (!(ok = mbar_wait_warp(&s_full[bj], phb, SITE_DC_SM_S))) break;
+      tc_fence_after();
+      // PV(j-1) is completion number (j-1)/NB of pv_done[(j-1)%NB]; S(j) completing implies PV(j-NB)
+      // done (S(j) was issued after it), so that barrier has at most this one phase pending.
+      const int jp = j > 0 ? j - 1 : 0;
+      if (!(ok = int_softmax_tile<GP>(rows, j, lane, wq, t, valid, scq, ks, vs, tS0 + bj * 16 + lane_off,
+                                      tO + lane_off, red_max, red_bar, &pv_done[jp % NB], (uint32_t)(jp / NB) & 1,
+                                      smem + C::OFF_P + bj * C::P_BYTES, C::RESCALE_THRESHOLD)))
+        break;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[bj]);
+    }
+    if (ok)
+      decode_epilogue<GP, false>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, 0, o_final,
+                                 0, nullptr);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

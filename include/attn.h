@@ -61,7 +61,12 @@ typedef enum {
   ATTN_ERR_INJECTED = 6     /* a host-side injected failure (tests of the error paths) */
 } attn_status_t;
 
-typedef enum { ATTN_BF16 = 0, ATTN_FP8_E4M3 = 1, ATTN_F32 = 2 } attn_dtype_t;
+/* Element types.  ATTN_INT8 / ATTN_INT4 are KV-cache codes only ([ORT-CPU] INT8/INT4 KV cache,
+ * V dequantised on the fly in the SV accumulation; the page gives no encoding, so the reading is
+ * two's complement with one float32 scale per (token, KV head)): INT8 one signed byte per element;
+ * INT4 two signed 4-bit elements per byte, element 2i in the low nibble of byte i, so a row of D
+ * elements is D/2 bytes. */
+typedef enum { ATTN_BF16 = 0, ATTN_FP8_E4M3 = 1, ATTN_F32 = 2, ATTN_INT8 = 3, ATTN_INT4 = 4 } attn_dtype_t;
 
 typedef struct {
   int B;       /* batch */
@@ -130,9 +135,13 @@ ATTN_API attn_status_t attn_prefill_varlen(const void* q, const void* k, const v
  * LSE = -inf.
  *
  *   q        device bf16 [B, Hq, D]
- *   k, v     device [B, Tmax, Hkv, D]: bf16 (kv_dtype = ATTN_BF16) or E4M3 codes (ATTN_FP8_E4M3)
- *   k_scale, v_scale  device float32 [B, Tmax, Hkv] dequantisation multipliers for FP8
- *            ([COOPT] Opt-KV FP8 cache); must be NULL for bf16.  Dequantised value = code * scale.
+ *   k, v     device [B, Tmax, Hkv, D]: bf16 (kv_dtype = ATTN_BF16), E4M3 codes (ATTN_FP8_E4M3) or
+ *            INT8 codes (ATTN_INT8); [B, Tmax, Hkv, D/2] packed INT4 codes (ATTN_INT4)
+ *   k_scale, v_scale  device float32 [B, Tmax, Hkv] dequantisation multipliers for the FP8 and
+ *            integer caches ([COOPT] Opt-KV FP8 cache, [ORT-CPU] INT8/INT4 cache); must be NULL for
+ *            bf16.  Dequantised value = code * scale.  Integer caches: |v_scale| is clamped to
+ *            [2^-100, 2^100] and |q| must stay below 2^114 (each query row is carried as f16
+ *            scaled by a power of two).
  *   kv_lens  device int32 [B], each in [0, Tmax]
  *   num_splits  0 = automatic (fills the GPU), else 1..4096
  *   o        device bf16 [B, Hq, D];  lse  device float32 [B, Hq] or NULL
@@ -159,7 +168,8 @@ ATTN_API attn_status_t attn_decode_splitkv(const void* q, const void* k, const v
  *
  *   q      device bf16 [B, n_q, Hq, D];  o device bf16 [B, n_q, Hq, D];  lse float32 [B, n_q, Hq]
  *   ws     at least attn_decode_multi_workspace_bytes(dims, Tmax, n_q, num_splits) bytes
- *   other arguments, layouts and errors as for attn_decode_splitkv
+ *   other arguments, layouts and errors as for attn_decode_splitkv, except that the cache is
+ *   bf16 or FP8: integer caches (ATTN_INT8, ATTN_INT4) give ATTN_ERR_UNSUPPORTED
  * ------------------------------------------------------------------------------------------ */
 ATTN_API size_t attn_decode_multi_workspace_bytes(attn_dims_t dims, int Tmax, int n_q, int num_splits);
 ATTN_API attn_status_t attn_decode_multi(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
@@ -178,8 +188,10 @@ ATTN_API attn_status_t attn_decode_multi(const void* q, const void* k, const voi
  * workspace rule as attn_decode_splitkv, with Tmax = max_pages * page_size.
  *
  *   q                 device bf16 [B, Hq, D]
- *   k_pool, v_pool    device [num_pages, page_size, Hkv, D]: bf16 or E4M3 codes (kv_dtype)
- *   k_scale_pool, v_scale_pool  device float32 [num_pages, page_size, Hkv] for FP8, else NULL
+ *   k_pool, v_pool    device [num_pages, page_size, Hkv, D]: bf16, E4M3 or INT8 codes (kv_dtype);
+ *                     [num_pages, page_size, Hkv, D/2] packed INT4 codes
+ *   k_scale_pool, v_scale_pool  device float32 [num_pages, page_size, Hkv] for the FP8 and integer
+ *                     caches, else NULL
  *   page_table        device int32 [B, max_pages]; entries used must lie in [0, num_pages)
  *   page_size         a multiple of 128 (a 128-token tile never straddles two pages)
  *   kv_lens           device int32 [B], each in [0, max_pages * page_size]

@@ -78,6 +78,8 @@ def test_prefill_empty_is_noop(L):
 
 @pytest.mark.parametrize("case", [
     dict(kv_dtype=1),                 # FP8 without scales
+    dict(kv_dtype=3), dict(kv_dtype=4),  # INT8 / INT4 without scales
+    dict(kv_dtype=2), dict(kv_dtype=5),  # not a cache element type
     dict(k_scale=FAKE),               # scales with bf16
     dict(kv_lens=None), dict(q=None), dict(Tmax=-1), dict(num_splits=-1), dict(num_splits=5000),
     dict(ws=None, num_splits=4),      # workspace required but missing
@@ -100,7 +102,8 @@ def test_decode_unsupported(L):
 @pytest.mark.parametrize("case", [
     dict(page_size=100), dict(page_size=64), dict(max_pages=0), dict(num_pages=0), dict(page_table=None),
     dict(k_pool=None), dict(q=None), dict(kv_lens=None), dict(kv_dtype=7), dict(k_scale=FAKE),
-    dict(kv_dtype=1), dict(ws=None), dict(num_splits=-1), dict(page_table=ctypes.c_void_p(0x10002)),
+    dict(kv_dtype=1), dict(kv_dtype=3), dict(kv_dtype=4), dict(ws=None), dict(num_splits=-1),
+    dict(page_table=ctypes.c_void_p(0x10002)),
 ])
 def test_decode_paged_invalid_args(L, case):
     a = dict(q=FAKE, k_pool=FAKE, v_pool=FAKE, kv_dtype=0, k_scale=None, v_scale=None, page_table=FAKE,
@@ -122,6 +125,13 @@ def test_decode_multi_invalid_args(L, case):
                              a["Tmax"], a["n_q"], a["dims"], a["num_splits"], a["o"], a["lse"], a["ws"], a["ws_bytes"],
                              None)
     assert st == 1
+
+
+@pytest.mark.parametrize("kv_dtype", [3, 4])
+def test_decode_multi_integer_cache_unsupported(L, kv_dtype):
+    st = L.attn_decode_multi(FAKE, FAKE, FAKE, kv_dtype, FAKE, FAKE, FAKE, 4096, 2, _dims(D=128), 4, FAKE, None, FAKE,
+                             1 << 30, None)
+    assert st == 2
 
 
 def test_decode_multi_rows_beyond_the_mma(L):
