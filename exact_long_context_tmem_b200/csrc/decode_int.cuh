@@ -18,16 +18,19 @@
 // so the probability that enters P, 2^(y - m) = 2^(x - m) * v_scale, stays below 2^threshold
 // whatever the scale; the row sum l adds 2^(x - m) = P / v_scale.
 //
-// Roles (480 threads, one CTA per (split, KV head, sequence)):
+// Roles (512 threads, one CTA per (split, KV head, sequence)):
 //   warp 0       TMA producer of the raw K code tiles (NCS-stage ring)
 //   warp 14      TMA producer of the raw V code tiles (NCS-stage ring)
-//   warp 1       TMEM allocator; lane 0 issues every MMA
+//   warp 1       TMEM allocator; lane 0 issues the S MMAs
+//   warp 15      lane 0 issues the PV MMAs
 //   warps 2..5   K converter: thread = token; codes -> f16 into TMEM
 //   warps 6..9   V converter: thread = token; codes -> f16 in shared memory (MN-major operand)
 //   warps 10..13 Q staging, softmax, epilogue: thread = token (later = output element d)
-// Scores, probabilities and converted tiles rotate through NB = 3 buffers: S(j+3) is issued right
-// after PV(j).  TMEM columns: S^T [0, 48) (three 16-column buffers), O^T [48, 64), converted K
-// [64, 256) (three 64-column buffers, 128 f16 per lane).
+// Issuing a tcgen05.mma costs its thread tens of cycles, so the S and PV chains (8 MMAs each per
+// tile) go to two threads, ordered only through barriers: S(j+NB) waits until the softmax has read
+// S(j) (s_free), and the softmax writes P(j+NB) once PV(j) has completed.  Scores, probabilities and
+// converted tiles rotate through NB = 3 buffers.  TMEM columns: S^T [0, 48) (three 16-column
+// buffers), O^T [48, 64), converted K [64, 256) (three 64-column buffers, 128 f16 per lane).
 #pragma once
 
 #include "decode.cuh"
@@ -54,9 +57,9 @@ struct DecodeIntCfg {
   static constexpr int OFF_RED = OFF_P + NB * P_BYTES;
   static constexpr int OFF_QSC = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;  // [16] 2^-e per query row
   static constexpr int OFF_BAR = OFF_QSC + 16 * 4;
-  static constexpr int N_BARS = 4 * NCS + 1 + 7 * NB + 1 + 2 + 1 + 1;
+  static constexpr int N_BARS = 4 * NCS + 1 + 8 * NB + 2 + 2 + 1 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
-  static constexpr int THREADS = 480;
+  static constexpr int THREADS = 512;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t COL_S = 0, COL_O = 48, COL_K = 64;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
@@ -120,6 +123,14 @@ __device__ __forceinline__ void int_row_half_to_f16(const uint8_t* tile, int t, 
   }
 }
 
+// One arrival per warp: every lane's prior writes (and the fences each lane issued) are ordered
+// before lane 0's release-arrive by the warp barrier.  Barriers fed this way count warps, which
+// keeps the same-address shared-memory atomics at one per warp instead of one per thread.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
 // Index of the (token, KV head) scale of sequence b's token tok, or -1 for an unmapped page.
 __device__ __forceinline__ long long int_scale_index(const DecodeParams& p, int b, int tok, int kvh) {
   long long page = b;
@@ -171,18 +182,26 @@ __device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kv
 // y = x + log2(v_scale): row maxima (warp redux, then the cross-warp exchange) -> lazy O rescale
 // -> this token's entries of P^T (2^(y - m), f16).  Returns false, warp-uniformly, if a bounded
 // wait ran out.  The parities follow decode_softmax_core.
+// S^T of the tile is read first and s_free is arrived on at once, so the next S into the same
+// buffer can be issued; the P^T buffer is written only after p_reuse (the PV that last read it, if
+// any) has completed.
 template <int GP>
 __device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, int lane, int wq, int t, bool valid,
                                                  const float (&scq)[GP], float ks, float vs, uint32_t tS_lane,
-                                                 uint32_t tO_lane, float* red_max, uint64_t* red_bar,
-                                                 uint64_t* prev_pv, uint32_t prev_pv_parity, uint8_t* p_tile,
-                                                 float threshold) {
+                                                 uint64_t* s_free, uint32_t tO_lane, float* red_max,
+                                                 uint64_t* red_bar, uint64_t* prev_pv, uint32_t prev_pv_parity,
+                                                 uint64_t* p_reuse, uint32_t p_reuse_parity, uint8_t* p_tile,
+                                                 float threshold, long long* evt_base_ = nullptr) {
   uint32_t sv[16];
   tmem_ld16(tS_lane, sv);
   tmem_wait_ld();
+  if (t == 0) ATTN_EVT(j, 10);
+  if (lane == 0 && j < 31) ATTN_EVT(32 + j, 4 + wq);
+  tc_fence_before();
+  warp_arrive(s_free, lane);
   const float avs = fminf(fmaxf(fabsf(vs), 0x1p-100f), 0x1p100f);
   const float lvs = __log2f(avs);
-  const float ivs = __frcp_rn(avs);
+  const float ivs = __fdividef(1.f, avs);
   const bool neg = vs < 0.f;
   float y[GP];
 #pragma unroll
@@ -193,8 +212,10 @@ __device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, in
     const float m = warp_max_redux(y[g]);
     if (lane == 0) rm[wq * 16 + g] = m;
   }
-  mbar_arrive(&red_bar[j & 1]);
+  if (lane == 0 && j < 31) ATTN_EVT(32 + j, wq);
+  warp_arrive(&red_bar[j & 1], lane);  // lane 0 wrote this warp's maxima
   if (!mbar_wait_warp(&red_bar[j & 1], (j >> 1) & 1, SITE_DC_SM_S)) return false;
+  if (t == 0) ATTN_EVT(j, 11);
   bool need = false;
   float alpha[GP];
 #pragma unroll
@@ -210,6 +231,7 @@ __device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, in
     }
   }
   if (need && j > 0) {  // rescale O^T row t once the previous PV is done
+    if (t == 0) ATTN_EVT(j, 14);
     if (!mbar_wait_warp(prev_pv, prev_pv_parity, SITE_DC_SM_O)) return false;
     tc_fence_after();
     uint32_t orow[16];
@@ -220,6 +242,8 @@ __device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, in
     tmem_st16(tO_lane, orow);
     tmem_wait_st();
   }
+  if (p_reuse && !mbar_wait_warp(p_reuse, p_reuse_parity, SITE_DC_SM_P)) return false;
+  if (t == 0) ATTN_EVT(j, 12);
   uint8_t* prow = p_tile + (t >> 6) * (16 * 128);
   const uint32_t pchunk = (t & 63) >> 3, pbyte = (t & 7) * 2;
 #pragma unroll
@@ -233,7 +257,7 @@ __device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, in
 }
 
 template <int GP, int BITS>
-__global__ void __launch_bounds__(480, 1)
+__global__ void __launch_bounds__(512, 1)
     decode_int_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
   using C = DecodeIntCfg<BITS>;
@@ -251,6 +275,11 @@ __global__ void __launch_bounds__(480, 1)
     decode_write_empty(p, G, split, kvh, b, threadIdx.x, blockDim.x);
     return;
   }
+#ifdef ATTN_PROF
+  // Event timeline of the grid's first CTA only (profile builds).
+  long long* const evt_base_ = (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) ? g_evt : nullptr;
+#endif
+  ATTN_EVT(63, 0);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -267,8 +296,9 @@ __global__ void __launch_bounds__(480, 1)
   uint64_t* kc_empty = kc_full + NB; // [NB] S MMA done reading it
   uint64_t* vc_full = kc_empty + NB; // [NB] converted V in shared memory
   uint64_t* vc_empty = vc_full + NB; // [NB] PV MMA done reading it
-  uint64_t* drain = vc_empty + NB;
-  uint64_t* red_bar = drain + 1;  // [2]
+  uint64_t* s_free = vc_empty + NB;  // [NB] the softmax has read S^T(j)
+  uint64_t* drain = s_free + NB;     // [2] each MMA issuer's own MMAs completed
+  uint64_t* red_bar = drain + 2;     // [2]
   uint64_t* sum_bar = red_bar + 2;
   uint64_t* o_final = sum_bar + 1;  // single phase: every PV of the split has completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_final + 1);
@@ -279,23 +309,25 @@ __global__ void __launch_bounds__(480, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NCS; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 128);
+      mbar_init(&k_empty[i], 4);
       mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 128);
+      mbar_init(&v_empty[i], 4);
     }
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, 4);
     for (int s = 0; s < NB; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 4);
       mbar_init(&pv_done[s], 1);
-      mbar_init(&kc_full[s], 128);
+      mbar_init(&kc_full[s], 4);
       mbar_init(&kc_empty[s], 1);
-      mbar_init(&vc_full[s], 128);
+      mbar_init(&vc_full[s], 4);
       mbar_init(&vc_empty[s], 1);
+      mbar_init(&s_free[s], 4);
     }
-    mbar_init(&red_bar[0], 128);
-    mbar_init(&red_bar[1], 128);
-    mbar_init(drain, 1);
+    mbar_init(&red_bar[0], 4);
+    mbar_init(&red_bar[1], 4);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     mbar_init(sum_bar, 128);
     mbar_init(o_final, 1);
     fence_barrier_init();
@@ -329,6 +361,7 @@ __global__ void __launch_bounds__(480, 1)
         const int page = pc.get(p, b, tok);
         mbar_arrive_expect_tx(&full[st], C::CODE_TILE);
         tma_load_4d(ring + st * C::CODE_TILE, tm, &full[st], 0, kvh, pc.offset(p, tok), page);
+        ATTN_EVT(j, is_k ? 0 : 1);
         issued = j + 1;
       }
       if (!ok)  // wait (bounded) for the copies still in flight before the CTA exits
@@ -336,56 +369,57 @@ __global__ void __launch_bounds__(480, 1)
           mbar_wait_drain(&full[j % C::NCS], (j / C::NCS) & 1, SITE_DC_DRAIN);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 15) {
+    // ------------------------------------------------------------------ MMA issuers (S: warp 1, PV: warp 15)
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = make_idesc_f16(128, 16, false, false, false);
-      constexpr uint32_t idesc_pv = make_idesc_f16(128, 16, true, false, false);
-      const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-      const uint32_t sP = smem_u32(smem + C::OFF_P);
-      const uint32_t sVc = smem_u32(smem + C::OFF_VC);
-      // S^T(j) [128 x 16] = K_j (TMEM, f16) . Q^T
-      auto issue_s = [&](int buf) {
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t qoff = (kk >> 2) * C::QBOX + (kk & 3) * 32;
-          mma_ts(tS0 + buf * 16, tK0 + buf * 64 + kk * 8, make_sdesc_sw128(sQ + qoff, 16, 1024), idesc_qk, kk > 0);
-        }
-      };
-      auto issue_pv = [&](int buf, bool acc) {  // O^T += V_j^T . P_j^T
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = make_sdesc_sw128(sVc + buf * C::VC_TILE + kk * 16 * 128, 128 * 128, 1024);
-          const uint64_t db = make_sdesc_sw128(sP + buf * C::P_BYTES + (kk >> 2) * C::PBOX + (kk & 3) * 32, 16, 1024);
-          mma_ss(tO, da, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(q_ready, 0, SITE_DC_MMA_K);
-      for (int jj = 0; jj < NB && jj < n && ok; ++jj) {
-        if (!(ok = mbar_wait(&kc_full[jj], 0, SITE_DC_MMA_K))) break;
-        tc_fence_after();
-        issue_s(jj);
-        mma_commit(&s_full[jj]);
-        mma_commit(&kc_empty[jj]);
-      }
-      for (int j = 0; j < n && ok; ++j) {
-        const int bj = j % NB;
-        const uint32_t ph = (j / NB) & 1;
-        if (!(ok = mbar_wait(&vc_full[bj], ph, SITE_DC_MMA_V))) break;
-        if (!(ok = mbar_wait(&p_full[bj], ph, SITE_DC_MMA_P))) break;
-        tc_fence_after();
-        issue_pv(bj, j > 0);
-        mma_commit(&pv_done[bj]);
-        mma_commit(&vc_empty[bj]);
-        if (j + NB < n) {  // S(j+NB) reuses buffer bj: S(j) was read before P(j) was published
-          if (!(ok = mbar_wait(&kc_full[bj], ph ^ 1, SITE_DC_MMA_K))) break;
+      bool ok = true;
+      if (warp == 1) {
+        // S^T(j) [128 x 16] = K_j (TMEM, f16) . Q^T
+        constexpr uint32_t idesc_qk = make_idesc_f16(128, 16, false, false, false);
+        const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+        ok = mbar_wait(q_ready, 0, SITE_DC_MMA_K);
+        for (int j = 0; j < n && ok; ++j) {
+          const int bj = j % NB;
+          const uint32_t ph = (j / NB) & 1;
+          if (!(ok = mbar_wait(&kc_full[bj], ph, SITE_DC_MMA_K))) break;
+          if (j >= NB && !(ok = mbar_wait(&s_free[bj], ph ^ 1, SITE_DC_MMA_S))) break;  // S(j-NB) read
           tc_fence_after();
-          issue_s(bj);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t qoff = (kk >> 2) * C::QBOX + (kk & 3) * 32;
+            mma_ts(tS0 + bj * 16, tK0 + bj * 64 + kk * 8, make_sdesc_sw128(sQ + qoff, 16, 1024), idesc_qk, kk > 0);
+          }
+          ATTN_EVT(j, 4);
           mma_commit(&s_full[bj]);
           mma_commit(&kc_empty[bj]);
         }
+        mma_commit(&drain[0]);
+        mbar_wait_drain(&drain[0], 0, SITE_DC_DRAIN);
+      } else {
+        // O^T += V_j^T . P_j^T
+        constexpr uint32_t idesc_pv = make_idesc_f16(128, 16, true, false, false);
+        const uint32_t sP = smem_u32(smem + C::OFF_P);
+        const uint32_t sVc = smem_u32(smem + C::OFF_VC);
+        for (int j = 0; j < n && ok; ++j) {
+          const int bj = j % NB;
+          const uint32_t ph = (j / NB) & 1;
+          ATTN_EVT(j, 8);
+          if (!(ok = mbar_wait(&vc_full[bj], ph, SITE_DC_MMA_V))) break;
+          ATTN_EVT(j, 9);
+          if (!(ok = mbar_wait(&p_full[bj], ph, SITE_DC_MMA_P))) break;
+          tc_fence_after();
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t da = make_sdesc_sw128(sVc + bj * C::VC_TILE + kk * 16 * 128, 128 * 128, 1024);
+            const uint64_t db = make_sdesc_sw128(sP + bj * C::P_BYTES + (kk >> 2) * C::PBOX + (kk & 3) * 32, 16, 1024);
+            mma_ss(tO, da, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          ATTN_EVT(j, 7);
+          mma_commit(&pv_done[bj]);
+          mma_commit(&vc_empty[bj]);
+        }
+        if (ok) mma_commit(o_final);
+        mma_commit(&drain[1]);
+        mbar_wait_drain(&drain[1], 0, SITE_DC_DRAIN);
       }
-      if (ok) mma_commit(o_final);
-      mma_commit(drain);
-      mbar_wait_drain(drain, 0, SITE_DC_DRAIN);
     }
     __syncwarp();
   } else if (warp < 6) {
@@ -410,9 +444,13 @@ __global__ void __launch_bounds__(480, 1)
         tmem_st32(tK0 + bj * 64 + half * 32 + lane_off, h);
       }
       tmem_wait_st();
-      mbar_arrive(&k_empty[st]);
       tc_fence_before();
-      mbar_arrive(&kc_full[bj]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&k_empty[st]);
+        mbar_arrive(&kc_full[bj]);
+      }
+      if (t == 0) ATTN_EVT(j, 2);
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------------ V converter warpgroup
@@ -436,9 +474,13 @@ __global__ void __launch_bounds__(480, 1)
           *reinterpret_cast<uint4*>(vc + half * (128 * 128) + sw128_offset(t, k)) =
               make_uint4(h[4 * k], h[4 * k + 1], h[4 * k + 2], h[4 * k + 3]);
       }
-      mbar_arrive(&v_empty[st]);
       fence_proxy_async_smem();
-      mbar_arrive(&vc_full[bj]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&v_empty[st]);
+        mbar_arrive(&vc_full[bj]);
+      }
+      if (t == 0) ATTN_EVT(j, 3);
     }
   } else {
     // ------------------------------------------------------------------ softmax warpgroup
@@ -450,8 +492,9 @@ __global__ void __launch_bounds__(480, 1)
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
     int_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, qsc);
     fence_proxy_async_smem();
-    mbar_arrive(q_ready);
+    warp_arrive(q_ready, lane);
     named_barrier_sync(1, 128);  // every row's 2^-e is in qsc
+    if (t == 0) ATTN_EVT(63, 1);
     float scq[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) scq[g] = p.scale_log2 * qsc[g];
@@ -463,14 +506,22 @@ __global__ void __launch_bounds__(480, 1)
       rows.l_part[g] = 0.f;
     }
     bool ok = true;
-    // Per-token scales are prefetched one tile ahead so their global-memory latency stays off
-    // the tile's critical path; an unmapped page leaves them at 1 (its codes land as zeros).
-    float ks_next = 1.f, vs_next = 1.f;
-    if (t0 + t < t1) {
-      const long long i = int_scale_index(p, b, t0 + t, kvh);
-      if (i >= 0) {
-        ks_next = __ldg(p.k_scale + i);
-        vs_next = __ldg(p.v_scale + i);
+    // Per-token scales are loaded SPF tiles ahead into a register ring: under full HBM streaming a
+    // plain global load takes longer than one tile, and the scores wait on k_scale.  An unmapped
+    // page leaves them at 1 (its codes land as zeros).
+    constexpr int SPF = 4;
+    float ksr[SPF], vsr[SPF];
+#pragma unroll
+    for (int i = 0; i < SPF; ++i) {
+      ksr[i] = 1.f;
+      vsr[i] = 1.f;
+      const int tk = t0 + i * 128 + t;
+      if (tk < t1) {
+        const long long x = int_scale_index(p, b, tk, kvh);
+        if (x >= 0) {
+          ksr[i] = __ldg(p.k_scale + x);
+          vsr[i] = __ldg(p.v_scale + x);
+        }
       }
     }
     for (int j = 0; j < n && ok; ++j) {
@@ -478,32 +529,50 @@ __global__ void __launch_bounds__(480, 1)
       const uint32_t phb = (j / NB) & 1;
       const int tok = t0 + j * 128 + t;
       const bool valid = tok < t1;
-      const float ks = ks_next, vs = vs_next;
-      ks_next = 1.f;
-      vs_next = 1.f;
-      if (tok + 128 < t1) {
-        const long long i = int_scale_index(p, b, tok + 128, kvh);
-        if (i >= 0) {
-          ks_next = __ldg(p.k_scale + i);
-          vs_next = __ldg(p.v_scale + i);
+      const float ks = ksr[0], vs = vsr[0];
+#pragma unroll
+      for (int i = 0; i + 1 < SPF; ++i) {
+        ksr[i] = ksr[i + 1];
+        vsr[i] = vsr[i + 1];
+      }
+      ksr[SPF - 1] = 1.f;
+      vsr[SPF - 1] = 1.f;
+      if (tok + SPF * 128 < t1) {
+        const long long x = int_scale_index(p, b, tok + SPF * 128, kvh);
+        if (x >= 0) {
+          ksr[SPF - 1] = __ldg(p.k_scale + x);
+          vsr[SPF - 1] = __ldg(p.v_scale + x);
         }
       }
+      if (t == 0) ATTN_EVT(j, 13);
+      if (lane == 0 && j < 31) ATTN_EVT(32 + j, 8 + wq);
       if (!(ok = mbar_wait_warp(&s_full[bj], phb, SITE_DC_SM_S))) break;
+      if (t == 0) ATTN_EVT(j, 5);
       tc_fence_after();
-      // PV(j-1) is completion number (j-1)/NB of pv_done[(j-1)%NB]; S(j) completing implies PV(j-NB)
-      // done (S(j) was issued after it), so that barrier has at most this one phase pending.
+      // PV(i) is completion number i/NB of pv_done[i%NB]; PV(j-1) and PV(j-NB) (the last reader of
+      // P buffer bj) are the oldest pending phases of their barriers, since PV(j) and later need
+      // this tile's P first, so each parity wait is unambiguous.
       const int jp = j > 0 ? j - 1 : 0;
       if (!(ok = int_softmax_tile<GP>(rows, j, lane, wq, t, valid, scq, ks, vs, tS0 + bj * 16 + lane_off,
-                                      tO + lane_off, red_max, red_bar, &pv_done[jp % NB], (uint32_t)(jp / NB) & 1,
-                                      smem + C::OFF_P + bj * C::P_BYTES, C::RESCALE_THRESHOLD)))
+                                      &s_free[bj], tO + lane_off, red_max, red_bar, &pv_done[jp % NB],
+                                      (uint32_t)(jp / NB) & 1, j >= NB ? &pv_done[bj] : nullptr, phb ^ 1,
+                                      smem + C::OFF_P + bj * C::P_BYTES, C::RESCALE_THRESHOLD
+#ifdef ATTN_PROF
+                                      , evt_base_
+#endif
+                                      )))
         break;
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[bj]);
+      warp_arrive(&p_full[bj], lane);
+      if (t == 0) ATTN_EVT(j, 6);
+      if (lane == 0 && j < 31) ATTN_EVT(32 + j, 12 + wq);
     }
+    if (t == 0) ATTN_EVT(63, 2);
     if (ok)
       decode_epilogue<GP, false>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, 0, o_final,
                                  0, nullptr);
+    if (t == 0) ATTN_EVT(63, 3);
   }
   tc_fence_before();
   __syncthreads();
