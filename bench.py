@@ -3,9 +3,10 @@
 
 Headline: causal GQA prefill, batch 2, 32 query / 8 KV heads, head dim 128, 8192 tokens,
 bf16 in / fp32 accumulate, in TFLOP/s (algorithmic FLOPs: the causal half only).  The same
-JSON line carries the split-KV decode workloads (ragged bf16 64K-128K cache; FP8 E4M3 cache,
-32768 tokens) in KV GB/s, each against the measured roofline, the oracle timed on the host
-cores, and an end-to-end number through host buffers.
+JSON line carries the split-KV decode workloads (ragged bf16 64K-128K cache; FP8 E4M3, INT8 and
+INT4 caches of 32768 tokens; paged and multi-token variants) in KV GB/s and the packed varlen
+prefill, each against the measured roofline, the oracle timed on the host cores, and an
+end-to-end number through host buffers.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--stream]
 

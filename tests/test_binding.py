@@ -1,0 +1,48 @@
+"""Host-side logic of the Python binding and of the benchmark's byte counts (no GPU)."""
+import re
+
+import pytest
+import torch
+
+import bench
+from exact_long_context_tmem_b200 import attn as A
+from exact_long_context_tmem_b200 import inputs as I
+
+
+def test_kv_kind_inference():
+    D = 128
+
+    def t(dtype, last=D):
+        return torch.empty((1, 1, 1, last), dtype=dtype)
+
+    assert A._kv_kind(t(torch.bfloat16), D, None) == A.ATTN_BF16
+    assert A._kv_kind(t(torch.uint8), D, None) == A.ATTN_FP8_E4M3
+    assert A._kv_kind(t(torch.float8_e4m3fn), D, None) == A.ATTN_FP8_E4M3
+    assert A._kv_kind(t(torch.int8), D, None) == A.ATTN_INT8
+    assert A._kv_kind(t(torch.uint8, D // 2), D, None) == A.ATTN_INT4  # packed rows of D/2 bytes
+    assert A._kv_kind(t(torch.uint8), D, "int8") == A.ATTN_INT8       # explicit name wins
+    with pytest.raises(KeyError):
+        A._kv_kind(t(torch.uint8), D, "int2")
+
+
+def test_binding_dtype_values_match_header():
+    src = open(A.os.path.join(A._PKG, "..", "include", "attn.h")).read()
+    enum = re.search(r"typedef enum \{([^}]*)\} attn_dtype_t;", src).group(1)
+    vals = {k: int(v) for k, v in re.findall(r"(ATTN_\w+)\s*=\s*(\d+)", enum)}
+    assert vals == {"ATTN_BF16": A.ATTN_BF16, "ATTN_FP8_E4M3": A.ATTN_FP8_E4M3, "ATTN_F32": A.ATTN_F32,
+                    "ATTN_INT8": A.ATTN_INT8, "ATTN_INT4": A.ATTN_INT4}
+
+
+@pytest.mark.parametrize("name,row", [("decode_b4_h32g8_d128_ragged64k_128k", 256),
+                                      ("decode_fp8_b16_h32g8_d128_t32768", 128),
+                                      ("decode_int8_b16_h32g8_d128_t32768", 128),
+                                      ("decode_int4_b16_h32g8_d128_t32768", 64)])
+def test_bench_decode_bytes(name, row):
+    """Algorithmic bytes: every visible token's K and V rows of every KV head (plus its two fp32
+    scales for a coded cache), Q and O in bf16 and the fp32 LSE."""
+    w = I.WORKLOADS[name]
+    lens = torch.tensor([1000, 0, 129] + [5] * (w.B - 3), dtype=torch.int32)
+    coded = w.kv_fp8 or w.kv_bits
+    per_tok = w.Hkv * (2 * row + (8 if coded else 0))
+    qo = w.B * w.Hq * (w.D * 2 * 2 + 4)
+    assert bench.decode_bytes(w, lens) == int(lens.sum()) * per_tok + qo
