@@ -46,12 +46,16 @@ L2_BYTES = 126 * 10**6
 # (profiles/*.md).  A value is reported only while the kernel's sources still hash to the ones
 # the counters were taken from; otherwise the traffic is unknown (null).
 NCU_TRAFFIC = {
-    "prefill": {"sources": ("ptx.cuh", "status.cuh", "prefill.cuh"), "sha1": "54e2a6b3e9999f5b",
-                "bytes": 392954112 + 112384768},
+    "prefill": {"sources": ("ptx.cuh", "status.cuh", "prefill.cuh"), "sha1": "3ceb15c1040336c2",
+                "bytes": 410138112 + 125584384},
     "decode_b4_h32g8_d128_ragged64k_128k": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh"),
-                                            "sha1": "192d79a32348f35a", "bytes": 1549363000 + 5569024},
+                                            "sha1": "91ba7351de606d2e", "bytes": 1549371648 + 1479424},
     "decode_fp8_b16_h32g8_d128_t32768": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh", "decode_fp8.cuh"),
-                                         "sha1": "6938565e5c0be643", "bytes": 1147849000 + 5528064},
+                                         "sha1": "a25edb49e6b129c4", "bytes": 1147812096 + 1815808},
+    "decode_int8_b16_h32g8_d128_t32768": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh", "decode_int.cuh"),
+                                          "sha1": "b7e3a3fe445590d3", "bytes": 1147757056 + 2215680},
+    "decode_int4_b16_h32g8_d128_t32768": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh", "decode_int.cuh"),
+                                          "sha1": "b7e3a3fe445590d3", "bytes": 608731136 + 2214912},
 }
 
 
