@@ -304,6 +304,7 @@ def bench_decode(name, steps, warmup, world, dev, pk, paged=False, n_q=1):
 
     w = I.WORKLOADS[name]
     d = I.decode_inputs(w)
+    d_contig = d
     lens = d["kv_lens"]
     Tmax = d["Tmax"]
     if paged:
@@ -355,7 +356,8 @@ def bench_decode(name, steps, warmup, world, dev, pk, paged=False, n_q=1):
                          "frac": round(gbs / pk["hbm_gbs"], 4),
                          "traffic": None if (paged or n_q > 1) else ncu_traffic(name),
                          "timed": "split kernel + merge kernel (one API call)"},
-            "launches": steps * (2 if splits > 1 else 1)}
+            "launches": steps * (2 if splits > 1 else 1),
+            "cpu_baseline": decode_oracle_sample(w, d_contig, n_q) if world == 1 else None}
 
 
 VARLEN = "prefill_varlen_b16_h32g8_d128_ragged512_2048"
@@ -392,7 +394,23 @@ def bench_prefill_varlen(steps, warmup, world, dev, pk):
     return {"workload": VARLEN, "value": round(tf * world, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
             "tokens": int(d["lens"].sum()), "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tf / pk["bf16_tflops"], 4), "traffic": None}, "launches": steps}
+                         "frac": round(tf / pk["bf16_tflops"], 4), "traffic": None}, "launches": steps,
+            "cpu_baseline": varlen_oracle_sample(w, d) if world == 1 else None}
+
+
+def varlen_oracle_sample(w, d):
+    """Time the float64 oracle on the first packed sequence of the varlen workload (all heads);
+    returns a cpu_baseline dict in TFLOP/s (causal pairs only, as the GPU line counts them)."""
+    from oracle import attention as O
+
+    n = int(d["lens"][0])
+    cu = torch.tensor([0, n], dtype=torch.int32)
+    t = time.perf_counter()
+    O.prefill_varlen(d["q"][:n], d["k"][:n], d["v"][:n], cu, cu, scale=w.scale, causal=True)
+    dt = time.perf_counter() - t
+    flops = 4.0 * w.D * w.Hq * n * (n + 1) / 2
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
+            "sample": f"sequence 0 of {w.B} ({n} tokens, {w.Hq} heads, {dt:.2f} s)"}
 
 
 def bench_stream(dev, pk):
@@ -443,6 +461,39 @@ def oracle_sample(w, n_rows, seed=4242):
     dt = time.perf_counter() - t
     flops = sum(4.0 * w.D * (r + 1) for r in rows) * w.B * w.Hq
     return flops / dt / 1e12, dt, rows
+
+
+def decode_oracle_sample(w, d, n_q=1):
+    """Time the float64 oracle on a bounded sample of a decode workload: sequence 0 of the cache
+    (every head; codes decoded to values first, as the oracle's input), single-token or n_q-token
+    decode.  Returns a cpu_baseline dict in the bench's unit (cache GB/s of the sample)."""
+    from oracle import attention as O
+
+    lens = d["kv_lens"][:1]
+    L = int(lens[0])
+    if w.kv_bits or w.kv_fp8:
+        if w.kv_bits:
+            from oracle import intq
+            dec = lambda c: intq.int_values(c[:1, :L], w.kv_bits)  # noqa: E731
+        else:
+            from oracle import fp8
+            dec = lambda c: fp8.e4m3_decode(c[:1, :L])  # noqa: E731
+        t = time.perf_counter()
+        k, v = dec(d["k_codes"]), dec(d["v_codes"])
+        ks, vs = d["k_scale"][:1, :L], d["v_scale"][:1, :L]
+    else:
+        t = time.perf_counter()
+        k, v, ks, vs = d["k"][:1, :L], d["v"][:1, :L], None, None
+    if n_q > 1:
+        q = I.randn_bf16((1, n_q, w.Hq, w.D), I.generator(w.seed + 11))
+        O.decode_multi(q, k, v, lens, scale=w.scale, k_scale=ks, v_scale=vs)
+    else:
+        O.decode(d["q"][:1], k, v, lens, scale=w.scale, k_scale=ks, v_scale=vs)
+    dt = time.perf_counter() - t
+    nb = L * (decode_bytes(w, torch.tensor([1])) - decode_bytes(w, torch.tensor([0])))
+    return {"value": round(nb / dt / 1e9, 3), "unit": "GB/s", "cores": host_threads(), "kind": "oracle",
+            "sample": f"sequence 0 of {w.B} ({L} tokens, {w.Hq} heads{f', {n_q} query tokens' if n_q > 1 else ''}), "
+                      f"contiguous cache, codes decoded inside the timed region ({dt:.2f} s)"}
 
 
 def main():

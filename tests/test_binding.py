@@ -46,3 +46,22 @@ def test_bench_decode_bytes(name, row):
     per_tok = w.Hkv * (2 * row + (8 if coded else 0))
     qo = w.B * w.Hq * (w.D * 2 * 2 + 4)
     assert bench.decode_bytes(w, lens) == int(lens.sum()) * per_tok + qo
+
+
+@pytest.mark.parametrize("kw,n_q", [({}, 1), ({"kv_fp8": True}, 1), ({"kv_bits": 8}, 1), ({"kv_bits": 4}, 1),
+                                    ({}, 3), ({"kv_fp8": True}, 2)])
+def test_bench_decode_oracle_sample(kw, n_q):
+    """The per-decode-line CPU baseline runs the oracle on sequence 0 of the same inputs."""
+    w = I.Workload("sample", "decode", B=3, Hq=8, Hkv=2, D=128, seed=3, **kw)
+    d = I.decode_inputs(w, lens=torch.tensor([300, 0, 17], dtype=torch.int32), Tmax=384)
+    cb = bench.decode_oracle_sample(w, d, n_q)
+    assert cb["kind"] == "oracle" and cb["unit"] == "GB/s" and cb["value"] > 0 and cb["cores"] >= 1
+    assert "300 tokens" in cb["sample"]
+
+
+def test_bench_varlen_oracle_sample():
+    w = I.Workload("sample_varlen", "prefill_varlen", B=3, Hq=4, Hkv=2, D=64, len_lo=40, len_hi=90, seed=9)
+    d = I.varlen_inputs(w)
+    cb = bench.varlen_oracle_sample(w, d)
+    assert cb["kind"] == "oracle" and cb["unit"] == "TFLOP/s" and cb["value"] > 0
+    assert f"{int(d['lens'][0])} tokens" in cb["sample"]
