@@ -121,6 +121,23 @@ def test_int_paged_matches_oracle_and_contiguous(cuda_device, bits, page_size):
     device_clean()
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+def test_int_bad_page_entry_reads_zeros_and_is_reported(cuda_device, bits):
+    """A table entry outside the pool is never dereferenced (its codes land as zeros through the
+    TMA's out-of-bounds fill, its scales are not read) and is reported by the status word."""
+    w, d = _case([1000], 1024, bits, seed=71)
+    pd = I.paged_inputs(d, 128, seed=4)
+    pd["page_table"][0, 2] = pd["num_pages"] + 5
+    dev = cuda_device
+    o, lse = A.attn_decode_paged(pd["q"].to(dev), pd["k_codes"].to(dev), pd["v_codes"].to(dev),
+                                 pd["page_table"].to(dev), pd["kv_lens"].to(dev), k_scale=pd["k_scale"].to(dev),
+                                 v_scale=pd["v_scale"].to(dev), num_splits=1)
+    torch.cuda.synchronize()
+    st, site = A.attn_device_status(reset=True)
+    assert st == A.ATTN_ERR_INVALID_ARG and site == 44
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
 def test_int_multi_token_unsupported(cuda_device):
     w, d = _case([300], 384, 8)
     q = d["q"][:, None].repeat(1, 2, 1, 1).contiguous().to(cuda_device)
