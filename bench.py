@@ -49,13 +49,13 @@ NCU_TRAFFIC = {
     "prefill": {"sources": ("ptx.cuh", "status.cuh", "prefill.cuh"), "sha1": "3ceb15c1040336c2",
                 "bytes": 410138112 + 125584384},
     "decode_b4_h32g8_d128_ragged64k_128k": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh"),
-                                            "sha1": "91ba7351de606d2e", "bytes": 1549371648 + 1479424},
+                                            "sha1": "49ce8af5a42b7165", "bytes": 1549371648 + 1479424},
     "decode_fp8_b16_h32g8_d128_t32768": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh", "decode_fp8.cuh"),
-                                         "sha1": "a25edb49e6b129c4", "bytes": 1147812096 + 1815808},
+                                         "sha1": "23caae74f340a143", "bytes": 1147812096 + 1815808},
     "decode_int8_b16_h32g8_d128_t32768": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh", "decode_int.cuh"),
-                                          "sha1": "b7e3a3fe445590d3", "bytes": 1147757056 + 2215680},
+                                          "sha1": "6d174515436707d9", "bytes": 1147757056 + 2215680},
     "decode_int4_b16_h32g8_d128_t32768": {"sources": ("ptx.cuh", "status.cuh", "decode.cuh", "decode_int.cuh"),
-                                          "sha1": "b7e3a3fe445590d3", "bytes": 608731136 + 2214912},
+                                          "sha1": "6d174515436707d9", "bytes": 608731136 + 2214912},
 }
 
 

@@ -7,17 +7,17 @@
 // One CTA = (split, KV head, sequence).  Per 128-token tile j:
 //   S^T_j [128 tokens x 16]  = K_j [128 x D] . Q^T [D x 16]        (G query rows, zero-padded to 16)
 //   O^T   [D x 16]          += V_j^T [D x 128] . P_j^T [128 x 16]
-// so every thread of the softmax warpgroup owns one token (one TMEM lane): per-token FP8
-// scales multiply that thread's score and probability, masking is a per-thread compare,
-// and only the G row maxima need a cross-thread reduction.  O^T rows are D, so the same
-// thread later owns output element d.
+// so every thread of the softmax warpgroup owns one token (one TMEM lane): per-token
+// dequantisation scales multiply that thread's score and probability, masking is a per-thread
+// compare, and only the G row maxima need a cross-thread reduction.  O^T rows are D, so the
+// same thread later owns output element d.
 //
-// FP8 E4M3 caches (LLM-CoOpt summary, "Opt-KV"): codes are converted to f16 in shared
-// memory (exact: every E4M3 value is an f16 value); the MMA then runs in f16, and Q is
-// carried as an f16 pair hi + lo (hi = f16(q), lo = f16(q - hi)) so that the score keeps
-// float32-level accuracy; the dequant scales never touch the MMA operands.
+// This file holds the bf16-cache kernel and what the decode kernels share (parameters, page
+// cursor, softmax steps, epilogue).  Coded caches have their own kernels: decode_fp8.cuh
+// (E4M3 codes fed to the MMA as they land) and decode_int.cuh (INT8 / INT4 codes widened to
+// f16 inside the tile load).
 //
-// Roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer,
+// Roles of the bf16 kernel (192 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer,
 // warps 2..5 softmax / epilogue (128 threads).  The query group is padded to GP (a power of two
 // <= 16, a template parameter) so the per-row loops unroll and run side by side.
 #pragma once
@@ -312,30 +312,6 @@ __device__ __forceinline__ void decode_stage_q(const DecodeParams& p, int G, int
     const int g = c >> 4, cc = c & 15;
     *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * (16 * 128) + sw128_offset(g, cc & 7)) =
         decode_q_chunk_load(p, G, kvh, b, c);
-  }
-}
-
-// Convert one token row (128 E4M3 codes, 128B-swizzled row `t` of the code tile) to f16 in the
-// two 64-wide boxes of the converted tile; invalid tokens become zeros.
-__device__ __forceinline__ void convert_row_e4m3(const uint8_t* codes_tile, uint8_t* f16_tile, int t, bool valid) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (valid) w = *reinterpret_cast<const uint4*>(codes_tile + sw128_offset(t, c));
-    const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-    uint32_t h[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      h[2 * i] = e4m3x2_to_f16x2((uint16_t)(wd[i] & 0xFFFFu));
-      h[2 * i + 1] = e4m3x2_to_f16x2((uint16_t)(wd[i] >> 16));
-    }
-    // codes 16c..16c+15 -> f16 chunks 2c, 2c+1 (8 elements each)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int chunk = 2 * c + e;
-      uint8_t* dst = f16_tile + (chunk >> 3) * (128 * 128) + sw128_offset(t, chunk & 7);
-      *reinterpret_cast<uint4*>(dst) = make_uint4(h[4 * e], h[4 * e + 1], h[4 * e + 2], h[4 * e + 3]);
-    }
   }
 }
 
