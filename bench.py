@@ -83,7 +83,9 @@ def peaks():
 
 # ------------------------------------------------------------------ distributed plumbing
 
-def dist_init(n_gpus):
+def dist_init(n_gpus, backend=None):
+    """One process per GPU under torchrun: NCCL with the device bound, or gloo (CPU plumbing
+    tests).  Returns (world, rank, local rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -91,9 +93,13 @@ def dist_init(n_gpus):
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        timeout = datetime.timedelta(seconds=300)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
     return world, rank, local
 
 
@@ -104,10 +110,12 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest of every rank's x (a device time): one all-reduce, on the GPU under NCCL."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
