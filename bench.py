@@ -471,6 +471,14 @@ def oracle_sample(w, n_rows, seed=4242):
     return flops / dt / 1e12, dt, rows
 
 
+def oracle_rates(w, n_rows, seconds, tflops):
+    """The oracle's sampled rate as query rows per second (each row over every batch and head),
+    and the time the whole prefill workload would take at the sample's FLOP rate (an
+    extrapolation, labelled as such: the oracle never runs the full configuration)."""
+    return {"rows_per_s": round(n_rows / seconds, 3),
+            "extrapolated_full_config_s": round(prefill_flops(w) / (tflops * 1e12), 1)}
+
+
 def decode_oracle_sample(w, d, n_q=1):
     """Time the float64 oracle on a bounded sample of a decode workload: sequence 0 of the cache
     (every head; codes decoded to values first, as the oracle's input), single-token or n_q-token
@@ -544,7 +552,8 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic N(0,1), seeded", "config": config, "impl": "reference",
                 "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                 "sample": f"{n_rows} sampled query rows x {w.B} batch x {w.Hq} heads per step"},
+                                 "sample": f"{n_rows} sampled query rows x {w.B} batch x {w.Hq} heads per step",
+                                 **oracle_rates(w, n_rows, statistics.mean(d for _, d in vals), value)},
                 "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -580,7 +589,8 @@ def main():
     if rank == 0 and world == 1:
         tf, dt, rows = oracle_sample(w, args.cpu_rows)
         cpu = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
-               "sample": f"{len(rows)} sampled query rows x {w.B} batch x {w.Hq} heads ({dt:.1f} s)"}
+               "sample": f"{len(rows)} sampled query rows x {w.B} batch x {w.Hq} heads ({dt:.1f} s)",
+               **oracle_rates(w, len(rows), dt, tf)}
     if rank == 0:
         line = {"metric": METRIC, "value": round(pre["tflops"], 2), "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["ms_per_step"], 4),

@@ -65,3 +65,10 @@ def test_bench_varlen_oracle_sample():
     cb = bench.varlen_oracle_sample(w, d)
     assert cb["kind"] == "oracle" and cb["unit"] == "TFLOP/s" and cb["value"] > 0
     assert f"{int(d['lens'][0])} tokens" in cb["sample"]
+
+
+def test_oracle_rates():
+    w = I.WORKLOADS["prefill_b2_h32g8_d128_s8192"]
+    r = bench.oracle_rates(w, 10, 2.0, 0.02)
+    assert r["rows_per_s"] == 5.0
+    assert abs(r["extrapolated_full_config_s"] - bench.prefill_flops(w) / 0.02e12) < 0.1

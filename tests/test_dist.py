@@ -71,3 +71,4 @@ def test_reference_arm_rank_gating():
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["rows_per_s"] > 0 and line["cpu_baseline"]["extrapolated_full_config_s"] > 0
