@@ -5,7 +5,8 @@
  *     O = softmax(scale * Q K^T + causal mask) V
  * with grouped-query heads, tile by tile with an online softmax so the S x T score
  * matrix never exists in memory; decode splits the key range into partials that a
- * log-sum-exp reduce merges exactly; a host streamer feeds (query block, key chunk)
+ * log-sum-exp reduce merges exactly, over bf16, FP8 E4M3, INT8 or INT4 caches (contiguous or
+ * paged) whose dequantisation happens inside the tile load; a host streamer feeds (query block, key chunk)
  * sub-tasks from pinned host memory under a device-memory budget and merges their
  * partials the same way.
  *
@@ -31,8 +32,9 @@
  *   - Layouts are row-major.  Q and O are token-major [B, S, Hq, D]; K and V are
  *     [B, T, Hkv, D]; the row log-sum-exp LSE is float32 [B, S, Hq] (same row order as O),
  *     natural log, including the score scale.  Query head h reads KV head h / (Hq / Hkv).
- *   - Supported: D in {64, 128}; bf16 Q/K/V; FP8 E4M3 K/V (decode); Hq % Hkv == 0;
- *     Hq / Hkv <= 16 for decode.  All base pointers 16-byte aligned.
+ *   - Supported: D in {64, 128}; bf16 Q/K/V; FP8 E4M3, INT8 and INT4 K/V codes with per-token
+ *     float32 scales (decode, D = 128); Hq % Hkv == 0; Hq / Hkv <= 16 for decode.  All base
+ *     pointers 16-byte aligned.
  *   - Thread safety: calls may be made from several host threads at once.
  */
 #ifndef ATTN_H_
