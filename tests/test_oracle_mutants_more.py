@@ -1,13 +1,15 @@
-"""Plant plausible mistakes in copies of the multi-token decode, packed varlen prefill and paged
-gather oracles (on the CPU) and check that their pins catch every one: a query position off by
-one, a lost causal mask, reversed tokens, top-left instead of bottom-right alignment, key ranges
-taken from the query offsets, a page index off by one, an ignored page table, a dropped partial
-page, a shifted slot offset."""
+"""Plant plausible mistakes in copies of the multi-token decode, packed varlen prefill, paged
+gather and streamed-decomposition oracles (on the CPU) and check that their pins catch every
+one: a query position off by one, a lost causal mask, reversed tokens, top-left instead of
+bottom-right alignment, key ranges taken from the query offsets, a page index off by one, an
+ignored page table, a dropped partial page, a shifted slot offset, a causal chunk test off by one
+or taken at the block's first row, and task offsets dropped."""
 import os
 import types
 
 import pytest
 
+from tests import test_oracle as TO
 from tests import test_oracle_multi as TM
 from tests import test_oracle_paged as TP
 from tests import test_oracle_varlen as TV
@@ -31,6 +33,12 @@ MUTANTS = {
                              "for i in range(n // page_size):"),
     "slot_offset_shifted": ("paged.py", "out[b, lo:hi] = pool[pg, : hi - lo]",
                             "out[b, lo:hi] = pool[pg, page_size - (hi - lo):]"),
+    # oracle/stream.py: the (query block, key chunk) decomposition
+    "chunk_test_off_by_one": ("stream.py", "if causal and kv_pos0 + kc > q_last:",
+                              "if causal and kv_pos0 + kc >= q_last:"),
+    "chunk_test_at_block_start": ("stream.py", "q_last = q_pos0 + min(S, qb + Bq) - 1", "q_last = q_pos0 + qb"),
+    "task_query_offset_dropped": ("stream.py", "q_pos0=qb, kv_pos0=kc)", "q_pos0=0, kv_pos0=kc)"),
+    "task_key_offset_dropped": ("stream.py", "q_pos0=qb, kv_pos0=kc)", "q_pos0=qb, kv_pos0=0)"),
 }
 
 
@@ -45,6 +53,10 @@ def _mutant(fname, old, new):
 
 def _pins(fname):
     """(test module, attribute the pins call the oracle through, pin callables)."""
+    if fname == "stream.py":
+        shapes = [(37, 8, 8), (64, 16, 32), (50, 50, 7), (9, 4, 16)]
+        return TO, "stream", [(lambda a=a, c=c: TO.test_stream_tasks_exact_cover(*a, c))
+                              for a in shapes for c in (True, False)] + [TO.test_stream_chunked_equals_unsplit]
     if fname == "paged.py":
         return TP, "PG", [TP.test_gather_by_hand, TP.test_swapped_entries_change_the_result,
                           TP.test_unmapped_page_below_length_is_an_error,
@@ -74,7 +86,7 @@ def test_pins_catch_mutant(name, monkeypatch):
 
 
 def test_unmutated_oracles_pass_the_same_pins():
-    for fname in ("attention.py", "paged.py"):
+    for fname in ("attention.py", "paged.py", "stream.py"):
         _, _, pins = _pins(fname)
         for pin in pins:
             pin()
