@@ -1,7 +1,7 @@
 """Build libattn.so in-tree: one nvcc invocation for sm_100a (kernels + C ABI + streamer).
 
 The CUDA runtime is linked statically, so the library carries its own runtime and shares
-only the driver's primary context with the caller (PyTorch or plain C).
+only the CUDA driver's primary context with the caller (PyTorch or plain C).
 """
 from __future__ import annotations
 

@@ -208,7 +208,7 @@ def test_stream_plan_fits_budget_and_config(L):
 ])
 def test_stream_tasks_exact_cover(L, S, chunk, budget, causal):
     """Every visible (query, key) pair lies in exactly one task rectangle (the oracle's
-    coverage counter is the judge)."""
+    coverage counter decides)."""
     plan = A.attn_stream_plan(1, 4, 2, 64, S, causal=causal, chunk_tokens=chunk, budget_bytes=budget)
     assert plan.device_bytes <= budget
     tasks = [A.attn_stream_task(plan, S, causal, i) for i in range(plan.n_tasks)]
