@@ -30,6 +30,8 @@ def _kv_kind(k, D: int, kv_dtype: str | None) -> int:
     INT8 codes; uint8 rows of D/2 bytes -> packed INT4 codes; uint8 / float8_e4m3fn rows of D -> E4M3
     codes; otherwise bf16."""
     if kv_dtype is not None:
+        if kv_dtype not in _KV_NAMES:
+            raise ValueError(f"kv_dtype must be one of {sorted(_KV_NAMES)}, not {kv_dtype!r}")
         return _KV_NAMES[kv_dtype]
     if k.dtype == torch.int8:
         return ATTN_INT8

@@ -21,7 +21,7 @@ def test_kv_kind_inference():
     assert A._kv_kind(t(torch.int8), D, None) == A.ATTN_INT8
     assert A._kv_kind(t(torch.uint8, D // 2), D, None) == A.ATTN_INT4  # packed rows of D/2 bytes
     assert A._kv_kind(t(torch.uint8), D, "int8") == A.ATTN_INT8       # explicit name wins
-    with pytest.raises(KeyError):
+    with pytest.raises(ValueError):
         A._kv_kind(t(torch.uint8), D, "int2")
 
 
