@@ -72,3 +72,17 @@ def test_oracle_rates():
     r = bench.oracle_rates(w, 10, 2.0, 0.02)
     assert r["rows_per_s"] == 5.0
     assert abs(r["extrapolated_full_config_s"] - bench.prefill_flops(w) / 0.02e12) < 0.1
+
+
+def test_cache_row_size_is_checked():
+    D = 128
+    ok8 = torch.empty((1, 4, 2, D), dtype=torch.int8)
+    A._check_kv_rows(ok8, ok8, D, A.ATTN_INT8)
+    ok4 = torch.empty((1, 4, 2, D // 2), dtype=torch.uint8)
+    A._check_kv_rows(ok4, ok4, D, A.ATTN_INT4)
+    with pytest.raises(ValueError):
+        A._check_kv_rows(ok8.view(torch.uint8), ok8.view(torch.uint8), D, A.ATTN_INT4)  # D bytes, not D/2
+    with pytest.raises(ValueError):
+        A._check_kv_rows(ok4, ok4, D, A.ATTN_FP8_E4M3)
+    with pytest.raises(ValueError):
+        A._check_kv_rows(ok8.transpose(1, 2), ok8, D, A.ATTN_INT8)  # not contiguous
