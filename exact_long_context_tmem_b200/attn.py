@@ -74,14 +74,20 @@ class StreamStats(ctypes.Structure):
 _lib = None
 
 
-def _check_kv_rows(k, v, D: int, kind: int):
-    """The library reads rows of D elements (D/2 bytes for packed INT4) with strides it derives
-    from the dimensions, so a cache tensor of another row size would be misread: refuse it."""
+def _check_kv_rows(k, v, D: int, kind: int, k_scale=None, v_scale=None):
+    """The library reads rows of D elements (D/2 bytes for packed INT4) and one float32 scale per
+    (token, KV head) with strides it derives from the dimensions, so a cache or scale tensor of
+    another shape, type or layout would be misread: refuse it."""
     row = D // 2 if kind == ATTN_INT4 else D
     for name, t in (("k", k), ("v", v)):
         if t.shape[-1] != row or not t.is_contiguous():
             raise ValueError(f"{name}: expected a contiguous cache with rows of {row} elements for this "
                              f"element type, got shape {tuple(t.shape)}")
+    for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        if t is not None and (tuple(t.shape) != tuple(k.shape[:-1]) or t.dtype != torch.float32
+                              or not t.is_contiguous()):
+            raise ValueError(f"{name}: expected contiguous float32 {tuple(k.shape[:-1])}, got "
+                             f"{t.dtype} {tuple(t.shape)}")
 
 
 def lib() -> ctypes.CDLL:
@@ -202,7 +208,7 @@ def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: 
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k, D, kv_dtype)
-    _check_kv_rows(k, v, D, kind)
+    _check_kv_rows(k, v, D, kind, k_scale, v_scale)
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -251,7 +257,7 @@ def attn_decode_multi(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: fl
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k, D, kv_dtype)
-    _check_kv_rows(k, v, D, kind)
+    _check_kv_rows(k, v, D, kind, k_scale, v_scale)
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, n_q, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -281,7 +287,7 @@ def attn_decode_paged(q, k_pool, v_pool, page_table, kv_lens, *, k_scale=None, v
     max_pages = page_table.shape[1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k_pool, D, kv_dtype)
-    _check_kv_rows(k_pool, v_pool, D, kind)
+    _check_kv_rows(k_pool, v_pool, D, kind, k_scale, v_scale)
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -313,7 +319,7 @@ def attn_decode_splitkv_noalloc(q, k, v, kv_lens, *, k_scale=None, v_scale=None,
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k, D, kv_dtype)
-    _check_kv_rows(k, v, D, kind)
+    _check_kv_rows(k, v, D, kind, k_scale, v_scale)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:

@@ -86,3 +86,14 @@ def test_cache_row_size_is_checked():
         A._check_kv_rows(ok4, ok4, D, A.ATTN_FP8_E4M3)
     with pytest.raises(ValueError):
         A._check_kv_rows(ok8.transpose(1, 2), ok8, D, A.ATTN_INT8)  # not contiguous
+
+
+def test_scale_shape_is_checked():
+    D = 128
+    k = torch.empty((2, 4, 3, D), dtype=torch.int8)
+    ok = torch.empty((2, 4, 3), dtype=torch.float32)
+    A._check_kv_rows(k, k, D, A.ATTN_INT8, ok, ok)
+    with pytest.raises(ValueError):
+        A._check_kv_rows(k, k, D, A.ATTN_INT8, ok.double(), ok)
+    with pytest.raises(ValueError):
+        A._check_kv_rows(k, k, D, A.ATTN_INT8, ok, torch.empty((2, 3, 4), dtype=torch.float32))
