@@ -42,9 +42,9 @@ DECODE_WORKLOADS = (("decode_bf16", "decode_b4_h32g8_d128_ragged64k_128k"),
 STREAM = "stream_b1_h32g8_d128_s1m_chunk64k"
 L2_BYTES = 126 * 10**6
 
-# DRAM bytes (read + write) per launch from one ncu capture of each kernel on its bench workload
-# (profiles/*.md).  A value is reported only while the kernel's sources still hash to the ones
-# the counters were taken from; otherwise the traffic is unknown (null).
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel on its bench workload.
+# A value is reported only while the kernel's sources still hash to the ones the counters were
+# taken from; otherwise the traffic is unknown (null).
 NCU_TRAFFIC = {
     "prefill": {"sources": ("ptx.cuh", "status.cuh", "prefill.cuh"), "sha1": "3ceb15c1040336c2",
                 "bytes": 410138112 + 125584384},

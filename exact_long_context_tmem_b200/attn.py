@@ -74,6 +74,24 @@ class StreamStats(ctypes.Structure):
 _lib = None
 
 
+def _expect(name, t, dtypes, shape):
+    """The library reads or writes exactly prod(shape) elements of one of `dtypes` at t's address,
+    row-major with no gaps.  A tensor of another type, shape or layout would be misread, or written
+    past its end on the device: refuse it.  None passes (optional outputs)."""
+    if t is None:
+        return
+    if not isinstance(dtypes, tuple):
+        dtypes = (dtypes,)
+    if t.dtype not in dtypes or tuple(t.shape) != tuple(int(x) for x in shape) or not t.is_contiguous():
+        want = "/".join(str(d).replace("torch.", "") for d in dtypes)
+        raise ValueError(f"{name}: expected a contiguous {want} tensor of shape {tuple(int(x) for x in shape)}, "
+                         f"got {str(t.dtype).replace('torch.', '')} {tuple(t.shape)}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+_ONE_BYTE = (torch.uint8, torch.int8, torch.float8_e4m3fn)
+
+
 def _check_kv_rows(k, v, D: int, kind: int, k_scale=None, v_scale=None):
     """The library reads rows of D elements (D/2 bytes for packed INT4) and one float32 scale per
     (token, KV head) with strides it derives from the dimensions, so a cache or scale tensor of
@@ -83,11 +101,31 @@ def _check_kv_rows(k, v, D: int, kind: int, k_scale=None, v_scale=None):
         if t.shape[-1] != row or not t.is_contiguous():
             raise ValueError(f"{name}: expected a contiguous cache with rows of {row} elements for this "
                              f"element type, got shape {tuple(t.shape)}")
+        ok = t.dtype == torch.bfloat16 if kind == ATTN_BF16 else t.dtype in _ONE_BYTE
+        if not ok:
+            raise ValueError(f"{name}: a {'bf16' if kind == ATTN_BF16 else 'one-byte code'} cache was expected "
+                             f"for this element kind, got {t.dtype}")
+    if tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"v: expected the shape of k {tuple(k.shape)}, got {tuple(v.shape)}")
     for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
         if t is not None and (tuple(t.shape) != tuple(k.shape[:-1]) or t.dtype != torch.float32
                               or not t.is_contiguous()):
             raise ValueError(f"{name}: expected contiguous float32 {tuple(k.shape[:-1])}, got "
                              f"{t.dtype} {tuple(t.shape)}")
+
+
+def _check_decode_io(q, kv_lens, o, lse, ws, q_shape, n_seq):
+    """Decode inputs and outputs: q bf16 [B, (n_q,) Hq, D], kv_lens int32 [B], o bf16 of q's shape,
+    lse float32 of q's shape without D, the workspace contiguous (its byte size is passed on)."""
+    B = q_shape[0]
+    _expect("q", q, torch.bfloat16, q_shape)
+    _expect("kv_lens", kv_lens, torch.int32, (B,))
+    _expect("o", o, torch.bfloat16, q_shape)
+    _expect("lse", lse, torch.float32, q_shape[:-1])
+    if n_seq is not None and n_seq != B:
+        raise ValueError(f"k/v: expected {B} sequences (the batch of q), got {n_seq}")
+    if ws is not None and not ws.is_contiguous():
+        raise ValueError("ws: expected a contiguous workspace")
 
 
 def lib() -> ctypes.CDLL:
@@ -99,7 +137,7 @@ def lib() -> ctypes.CDLL:
         raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_long_context_tmem_b200.build`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i, ll, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t, ctypes.c_float
-    L.attn_prefill.argtypes = [vp, vp, vp, vp, i, vp, Dims, i, i, i, ll, ll, vp]
+    L.attn_prefill.argtypes = [vp, vp, vp, vp, i, vp, Dims, i, i, i, ll, ll, ctypes.POINTER(ll), vp]
     L.attn_prefill.restype = i
     L.attn_decode_workspace_bytes.argtypes = [Dims, i, i]
     L.attn_decode_workspace_bytes.restype = sz
@@ -171,10 +209,25 @@ def _need_cuda(*ts):
             raise ValueError("device tensors expected (the library runs on the GPU only)")
 
 
+def _bshd_strides(name, t, dtypes, shape):
+    """Element strides (batch, token, head) of a [B, S, H, D] view whose D elements are contiguous,
+    as attn_prefill takes them; the view may be a slice of a larger tensor (fused QKV, a subset of
+    heads, a [B, H, S, D] tensor transposed)."""
+    if t.dtype not in dtypes or tuple(t.shape) != tuple(shape):
+        want = "/".join(str(d).replace("torch.", "") for d in dtypes)
+        raise ValueError(f"{name}: expected a {want} tensor of shape {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+    if t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name}: the last (D) dimension must be contiguous, got strides {t.stride()}")
+    return [t.stride(0), t.stride(1), t.stride(2)]
+
+
 def attn_prefill(q, k, v, *, causal: bool = True, scale: float | None = None, q_pos0: int = 0, kv_pos0: int = 0,
                  o=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True, stream=None):
-    """q [B,S,Hq,D], k/v [B,T,Hkv,D] bf16 CUDA tensors -> (o [B,S,Hq,D], lse [B,S,Hq] float32)."""
-    _need_cuda(q, k, v)
+    """q [B,S,Hq,D], k/v [B,T,Hkv,D] bf16 CUDA tensors -> (o [B,S,Hq,D], lse [B,S,Hq] float32).
+
+    q, k, v and a caller-supplied o may be strided views (D contiguous, every other stride a
+    multiple of 16 bytes): they are read and written in place through attn_prefill's strides."""
+    _need_cuda(q, k, v, o, lse)
     B, S, Hq, D = q.shape
     T, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
@@ -182,9 +235,16 @@ def attn_prefill(q, k, v, *, causal: bool = True, scale: float | None = None, q_
         o = torch.empty((B, S, Hq, D), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
+    _expect("lse", lse, torch.float32, (B, S, Hq))
+    bf = (torch.bfloat16,)
+    st_all = (_bshd_strides("q", q, bf, (B, S, Hq, D)) + _bshd_strides("k", k, bf, (B, T, Hkv, D)) +
+              _bshd_strides("v", v, bf, (B, T, Hkv, D)) +
+              _bshd_strides("o", o, (torch.bfloat16, torch.float32), (B, S, Hq, D)))
+    packed = all(t.is_contiguous() for t in (q, k, v, o))
+    strides = None if packed else (ctypes.c_longlong * 12)(*st_all)
     od = ATTN_F32 if o.dtype == torch.float32 else ATTN_BF16
     st = lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), od, _ptr(lse), _dims(B, Hq, Hkv, D, scale), S, T,
-                            int(bool(causal)), int(q_pos0), int(kv_pos0), _stream(stream))
+                            int(bool(causal)), int(q_pos0), int(kv_pos0), strides, _stream(stream))
     _check(st, "attn_prefill")
     return o, lse
 
@@ -203,12 +263,13 @@ def attn_decode_splitkv(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: 
     """q [B,Hq,D] bf16; k/v [B,Tmax,Hkv,D] bf16, uint8 E4M3 codes or int8 codes, or [B,Tmax,Hkv,D/2]
     uint8 packed INT4 codes (+ float32 scales [B,Tmax,Hkv] for every coded cache); kv_lens int32
     [B] on the device -> (o [B,Hq,D] bf16, lse [B,Hq] float32)."""
-    _need_cuda(q, k, v, kv_lens, k_scale, v_scale)
+    _need_cuda(q, k, v, kv_lens, k_scale, v_scale, o, lse, ws)
     B, Hq, D = q.shape
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k, D, kv_dtype)
     _check_kv_rows(k, v, D, kind, k_scale, v_scale)
+    _check_decode_io(q, kv_lens, o, lse, ws, (B, Hq, D), k.shape[0])
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -230,11 +291,18 @@ def attn_prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, 
                         out_dtype=torch.bfloat16, stream=None):
     """Packed batch: q [total_q,Hq,D], k/v [total_k,Hkv,D] bf16; cu_seqlens_q/k int32 [B+1] on the
     device -> (o [total_q,Hq,D], lse [total_q,Hq] float32)."""
-    _need_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    _need_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k, o, lse)
     total_q, Hq, D = q.shape
     total_k, Hkv = k.shape[0], k.shape[1]
     B = cu_seqlens_q.shape[0] - 1
     scale = 1.0 / math.sqrt(D) if scale is None else scale
+    _expect("q", q, torch.bfloat16, (total_q, Hq, D))
+    _expect("k", k, torch.bfloat16, (total_k, Hkv, D))
+    _expect("v", v, torch.bfloat16, (total_k, Hkv, D))
+    _expect("cu_seqlens_q", cu_seqlens_q, torch.int32, (B + 1,))
+    _expect("cu_seqlens_k", cu_seqlens_k, torch.int32, (B + 1,))
+    _expect("o", o, (torch.bfloat16, torch.float32), (total_q, Hq, D))
+    _expect("lse", lse, torch.float32, (total_q, Hq))
     if o is None:
         o = torch.empty((total_q, Hq, D), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
@@ -252,12 +320,13 @@ def attn_decode_multi(q, k, v, kv_lens, *, k_scale=None, v_scale=None, scale: fl
                       kv_dtype: str | None = None):
     """q [B,n_q,Hq,D] bf16 (n_q new tokens per sequence, already in the cache); k/v as for
     attn_decode_splitkv -> (o [B,n_q,Hq,D] bf16, lse [B,n_q,Hq] float32)."""
-    _need_cuda(q, k, v, kv_lens, k_scale, v_scale)
+    _need_cuda(q, k, v, kv_lens, k_scale, v_scale, o, lse, ws)
     B, n_q, Hq, D = q.shape
     Tmax, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k, D, kv_dtype)
     _check_kv_rows(k, v, D, kind, k_scale, v_scale)
+    _check_decode_io(q, kv_lens, o, lse, ws, (B, n_q, Hq, D), k.shape[0])
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, n_q, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -281,13 +350,17 @@ def attn_decode_paged(q, k_pool, v_pool, page_table, kv_lens, *, k_scale=None, v
     or [num_pages, page_size, Hkv, D/2] packed INT4 codes (+ float32 scale pools
     [num_pages, page_size, Hkv] for every coded cache); page_table int32 [B, max_pages] and
     kv_lens int32 [B] on the device -> (o [B,Hq,D] bf16, lse [B,Hq] float32)."""
-    _need_cuda(q, k_pool, v_pool, page_table, kv_lens, k_scale, v_scale)
+    _need_cuda(q, k_pool, v_pool, page_table, kv_lens, k_scale, v_scale, o, lse, ws)
     B, Hq, D = q.shape
     num_pages, page_size, Hkv = k_pool.shape[0], k_pool.shape[1], k_pool.shape[2]
+    if page_table.dim() != 2:
+        raise ValueError(f"page_table: expected int32 [B, max_pages], got shape {tuple(page_table.shape)}")
     max_pages = page_table.shape[1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k_pool, D, kv_dtype)
     _check_kv_rows(k_pool, v_pool, D, kind, k_scale, v_scale)
+    _check_decode_io(q, kv_lens, o, lse, ws, (B, Hq, D), None)
+    _expect("page_table", page_table, torch.int32, (B, max_pages))
     dims = _dims(B, Hq, Hkv, D, scale)
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
@@ -320,6 +393,7 @@ def attn_decode_splitkv_noalloc(q, k, v, kv_lens, *, k_scale=None, v_scale=None,
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     kind = _kv_kind(k, D, kv_dtype)
     _check_kv_rows(k, v, D, kind, k_scale, v_scale)
+    _check_decode_io(q, kv_lens, o, lse, None, (B, Hq, D), k.shape[0])
     if o is None:
         o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -337,6 +411,10 @@ def attn_merge_lse(o_parts, lse_parts, *, o_out=None, lse_out=None, accumulate: 
     """o_parts float32 [P,R,D], lse_parts float32 [P,R] -> (o_out [R,D], lse_out [R])."""
     _need_cuda(o_parts, lse_parts, o_out, lse_out)
     P, R, D = o_parts.shape
+    _expect("o_parts", o_parts, torch.float32, (P, R, D))
+    _expect("lse_parts", lse_parts, torch.float32, (P, R))
+    _expect("o_out", o_out, (torch.float32, torch.bfloat16), (R, D))
+    _expect("lse_out", lse_out, torch.float32, (R,))
     if o_out is None:
         o_out = torch.empty((R, D), dtype=out_dtype, device=o_parts.device)
     if lse_out is None:
@@ -374,6 +452,14 @@ def attn_chunked_stream(q_h, k_h, v_h, *, causal=True, chunk_tokens=0, budget_by
     B, S, Hq, D = q_h.shape
     Hkv = k_h.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
+    for t in (o_h, lse_h):
+        if t is not None and t.is_cuda:
+            raise ValueError("attn_chunked_stream takes host tensors")
+    _expect("q_h", q_h, torch.bfloat16, (B, S, Hq, D))
+    _expect("k_h", k_h, torch.bfloat16, (B, S, Hkv, D))
+    _expect("v_h", v_h, torch.bfloat16, (B, S, Hkv, D))
+    _expect("o_h", o_h, torch.bfloat16, (B, S, Hq, D))
+    _expect("lse_h", lse_h, torch.float32, (B, S, Hq))
     if o_h is None:
         o_h = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, pin_memory=True)
     if lse_h is None and want_lse:

@@ -6,6 +6,7 @@ only the CUDA driver's primary context with the caller (PyTorch or plain C).
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -15,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libattn.so")
 SOURCES = ["api.cu", "stream.cpp"]
-HEADERS = ["ptx.cuh", "status.cuh", "prefill.cuh", "decode.cuh", "decode_fp8.cuh", "merge.cuh"]
+_INCLUDE = re.compile(r'^\s*#\s*include\s+"([^"]+)"', re.M)
 
 
 def nvcc() -> str:
@@ -25,11 +26,24 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libattn.so")
 
 
+def dependencies():
+    """Every file the library is built from: the sources and, transitively, each file they
+    include with quotes (so an edited header always triggers a rebuild)."""
+    seen = []
+    todo = [os.path.join(CSRC, s) for s in SOURCES]
+    while todo:
+        f = os.path.normpath(todo.pop())
+        if f in seen:
+            continue
+        seen.append(f)
+        with open(f) as fh:
+            for inc in _INCLUDE.findall(fh.read()):
+                todo.append(os.path.join(os.path.dirname(f), inc))
+    return sorted(seen)
+
+
 def _inputs():
-    files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
-    files.append(os.path.join(ROOT, "include", "attn.h"))
-    files.append(os.path.abspath(__file__))
-    return files
+    return dependencies() + [os.path.abspath(__file__)]
 
 
 def up_to_date() -> bool:

@@ -57,14 +57,19 @@ static EncodeTiledFn encode_fn() {
 
 // 4-D tiled map over a row-major [d3][d2][d1][d0] tensor, 128-byte swizzle (or `swz`), zero fill out
 // of bounds.
+// A 4-D tiled map over (D, heads, tokens, batch).  `strides` gives the element strides of the
+// three outer dimensions (NULL: packed row-major, as the dimensions imply).
 static attn_status_t make_map_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes,
                                  const uint64_t dims[4], const uint32_t box[4],
-                                 CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+                                 CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B,
+                                 const long long* strides = nullptr) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t gdim[4] = {dims[0], dims[1], dims[2], dims[3]};
   cuuint64_t gstride[3] = {dims[0] * elem_bytes, dims[0] * dims[1] * elem_bytes,
                            dims[0] * dims[1] * dims[2] * elem_bytes};
+  if (strides)
+    for (int i = 0; i < 3; ++i) gstride[i] = (cuuint64_t)strides[i] * (cuuint64_t)elem_bytes;
   cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
   cuuint32_t es[4] = {1, 1, 1, 1};
   CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
@@ -100,11 +105,13 @@ static constexpr float kLog2e = 1.4426950408889634f;
 // Dense batch: q [B, S, Hq, D], k/v [B, T, Hkv, D].  Packed batch (cu_q non-null): q/o/lse rows
 // [total_q] and k/v rows [total_k] (S = total_q, T = total_k, a single TMA batch), the sequences
 // cut by the device cumulative lengths, and max_s the longest query count (grid size).
+// strides: NULL (packed [B, S, H, D] tensors) or 12 element strides, (batch, token, head) for
+// q, k, v and o in that order; already validated.
 template <int D>
 static attn_status_t launch_prefill(const void* q, const void* k, const void* v, void* o, int o_f32, float* lse,
                                     const attn_dims_t& d, int S, int T, int causal, long long q_pos0,
                                     long long kv_pos0, cudaStream_t stream, const int* cu_q = nullptr,
-                                    const int* cu_k = nullptr, int max_s = 0) {
+                                    const int* cu_k = nullptr, int max_s = 0, const long long* strides = nullptr) {
   using C = PrefillCfg<D>;
   static std::atomic<uint64_t> smem_done{0};
   attn_status_t st = ensure_smem(prefill_fwd_sm100<D>, C::SMEM_BYTES, smem_done);
@@ -114,9 +121,22 @@ static attn_status_t launch_prefill(const void* q, const void* k, const void* v,
   const uint64_t dq[4] = {(uint64_t)D, (uint64_t)d.Hq, (uint64_t)std::max(S, 1), nb};
   const uint64_t dk[4] = {(uint64_t)D, (uint64_t)d.Hkv, (uint64_t)std::max(T, 1), nb};
   const uint32_t box[4] = {64, 1, 128, 1};
-  if ((st = make_map_4d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dq, box)) != ATTN_OK) return st;
-  if ((st = make_map_4d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box)) != ATTN_OK) return st;
-  if ((st = make_map_4d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box)) != ATTN_OK) return st;
+  // The map's outer strides run (head, token, batch); the argument lists (batch, token, head).
+  long long sq[3], sk[3], sv[3];
+  if (strides) {
+    for (int i = 0; i < 3; ++i) {
+      sq[i] = strides[2 - i];
+      sk[i] = strides[5 - i];
+      sv[i] = strides[8 - i];
+    }
+  }
+  const CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B;
+  if ((st = make_map_4d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dq, box, swz, strides ? sq : nullptr)) != ATTN_OK)
+    return st;
+  if ((st = make_map_4d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box, swz, strides ? sk : nullptr)) != ATTN_OK)
+    return st;
+  if ((st = make_map_4d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, box, swz, strides ? sv : nullptr)) != ATTN_OK)
+    return st;
   PrefillParams p{};
   p.B = d.B;
   p.Hq = d.Hq;
@@ -138,6 +158,9 @@ static attn_status_t launch_prefill(const void* q, const void* k, const void* v,
   p.n_items = (int)items;
   p.o = o;
   p.o_f32 = o_f32;
+  p.o_sb = strides ? strides[9] : (long long)S * d.Hq * D;
+  p.o_ss = strides ? strides[10] : (long long)d.Hq * D;
+  p.o_sh = strides ? strides[11] : (long long)D;
   p.lse = lse;
   p.cu_q = cu_q;
   p.cu_k = cu_k;
@@ -401,17 +424,35 @@ const char* attn_status_string(attn_status_t s) {
 
 int attn_last_cuda_error(void) { return t_last_cuda_error; }
 
+// The 12 element strides of attn_prefill: each positive, a whole number of 16-byte units (TMA
+// strides and the 16-byte output stores need it) and below TMA's 2^40-byte stride limit.
+static bool prefill_strides_ok(const long long* s, int o_f32) {
+  for (int i = 0; i < 12; ++i) {
+    const long long unit = (i >= 9 && o_f32) ? 4 : 8;  // elements per 16 bytes
+    if (s[i] <= 0 || s[i] % unit != 0 || s[i] >= (1LL << 38)) return false;
+  }
+  return true;
+}
+
 attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o, attn_dtype_t o_dtype, float* lse,
                            attn_dims_t dims, int S, int T, int causal, long long q_pos0, long long kv_pos0,
-                           void* stream) {
+                           const long long* strides, void* stream) {
   if (!dims_ok(dims) || S < 0 || T < 0 || q_pos0 < 0 || kv_pos0 < 0) return ATTN_ERR_INVALID_ARG;
   if (o_dtype != ATTN_BF16 && o_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  if (strides && !prefill_strides_ok(strides, o_dtype == ATTN_F32)) return ATTN_ERR_INVALID_ARG;
   if (dims.B == 0 || S == 0) return ATTN_OK;
   if (!q || !o || (T > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || (T > 0 && (!aligned16(k) || !aligned16(v))) || (lse && !aligned4(lse)))
     return ATTN_ERR_INVALID_ARG;
   if (dims.D != 64 && dims.D != 128) return ATTN_ERR_UNSUPPORTED;
-  if (T == 0) {
+  long long s_nokv[12];
+  if (T == 0 && strides) {
+    // No keys and a strided output: the kernel itself writes the empty rows (O = 0, LSE = -inf)
+    // and never reads a key; its K/V maps only need a valid base, so they point at q.
+    for (int i = 0; i < 12; ++i) s_nokv[i] = strides[i < 9 ? i % 3 : i];
+    k = v = q;
+    strides = s_nokv;
+  } else if (T == 0) {
     // No keys: every row is empty.  O = 0, LSE = -inf, written by the merge kernel with no parts.
     MergeParams mp{};
     mp.P = 0;
@@ -430,8 +471,11 @@ attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o,
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int f32 = o_dtype == ATTN_F32;
-  if (dims.D == 128) return launch_prefill<128>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st);
-  return launch_prefill<64>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st);
+  if (dims.D == 128)
+    return launch_prefill<128>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st, nullptr, nullptr, 0,
+                               strides);
+  return launch_prefill<64>(q, k, v, o, f32, lse, dims, S, T, causal, q_pos0, kv_pos0, st, nullptr, nullptr, 0,
+                            strides);
 }
 
 attn_status_t attn_prefill_varlen(const void* q, const void* k, const void* v, void* o, attn_dtype_t o_dtype,
@@ -480,13 +524,20 @@ size_t attn_decode_workspace_bytes(attn_dims_t dims, int Tmax, int num_splits) {
   return decode_ws_bytes(dims, decode_splits(dims, Tmax, num_splits));
 }
 
-attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
-                                  const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax,
-                                  attn_dims_t dims, int num_splits, void* o, float* lse, void* ws, size_t ws_bytes,
-                                  void* stream) {
+}  // extern "C"
+
+// Every check of attn_decode_splitkv that does not involve the workspace, in its order.  ATTN_OK
+// with *empty set means a valid call with nothing to do (B = 0).
+static attn_status_t decode_splitkv_args(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                         const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax,
+                                         const attn_dims_t& dims, int num_splits, void* o, float* lse, bool* empty) {
+  *empty = false;
   if (!dims_ok(dims) || Tmax < 0 || num_splits < 0 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
   if (!kv_dtype_ok(kv_dtype)) return ATTN_ERR_INVALID_ARG;
-  if (dims.B == 0) return ATTN_OK;
+  if (dims.B == 0) {
+    *empty = true;
+    return ATTN_OK;
+  }
   if (!q || !o || !kv_lens || (Tmax > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
   const bool quant = kv_dtype != ATTN_BF16;  // codes + per-token scales
   if (quant != (k_scale != nullptr) || quant != (v_scale != nullptr)) return ATTN_ERR_INVALID_ARG;
@@ -495,6 +546,19 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, a
   if (quant && (!aligned4(k_scale) || !aligned4(v_scale))) return ATTN_ERR_INVALID_ARG;
   if (dims.D != 128 || dims.Hq / dims.Hkv > 16) return ATTN_ERR_UNSUPPORTED;
   if (dims.B > 65535 || dims.Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+extern "C" {
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
+                                  const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax,
+                                  attn_dims_t dims, int num_splits, void* o, float* lse, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  bool empty = false;
+  const attn_status_t a = decode_splitkv_args(q, k, v, kv_dtype, k_scale, v_scale, kv_lens, Tmax, dims, num_splits,
+                                              o, lse, &empty);
+  if (a != ATTN_OK || empty) return a;
   const int P = decode_splits(dims, Tmax, num_splits);
   const size_t need = decode_ws_bytes(dims, P);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return ATTN_ERR_INVALID_ARG;
@@ -568,29 +632,63 @@ attn_status_t attn_decode_multi(const void* q, const void* k, const void* v, att
 // Split-KV decode without allocation: the split partials live in this static device array
 // (ATTN_NOALLOC_SCRATCH_BYTES per device, held until the process exits).  Host code must not pass
 // the array's name to a kernel — on the host it is only a stand-in — so its device address is
-// looked up once per device with cudaGetSymbolAddress, with that device current.
+// looked up with cudaGetSymbolAddress, with the device current, once per device and context: the
+// address is cached with the context it belongs to, and looked up again if the device's context
+// changes (after a cudaDeviceReset the module, and with it the array, is loaded anew).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+static attn_status_t noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  static CUcontext owner[64] = {};
+  int dev = 0;
+  ATTN_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return ATTN_ERR_UNSUPPORTED;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  if (!get) return cuda_fail(cudaErrorNotSupported);
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) ctx = nullptr;  // none yet: the lookup below makes it current
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ctx || !addr[dev] || owner[dev] != ctx) {
+    void* p = nullptr;
+    ATTN_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return cuda_fail(cudaErrorNotSupported);
+    addr[dev] = p;
+    owner[dev] = ctx;
+  }
+  *out = addr[dev];
+  return ATTN_OK;
+}
 
 attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* k, const void* v, attn_dtype_t kv_dtype,
                                           const float* k_scale, const float* v_scale, const int* kv_lens, int Tmax,
                                           attn_dims_t dims, int num_splits, void* o, float* lse, void* stream) {
-  if (!dims_ok(dims) || Tmax < 0 || num_splits < 0 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
+  // Argument checks first, in attn_decode_splitkv's order; the scratch limit after them.
+  bool empty = false;
+  const attn_status_t a = decode_splitkv_args(q, k, v, kv_dtype, k_scale, v_scale, kv_lens, Tmax, dims, num_splits,
+                                              o, lse, &empty);
+  if (a != ATTN_OK || empty) return a;
   const size_t need = decode_ws_bytes(dims, decode_splits(dims, Tmax, num_splits));
   if (need > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_BUDGET;
   void* ws = nullptr;
   if (need > 0) {
-    static std::mutex mu;
-    static void* scratch[64] = {};
-    int dev = 0;
-    ATTN_CUDA(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 64) return ATTN_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!scratch[dev]) {
-      void* p = nullptr;
-      ATTN_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-      scratch[dev] = p;
-    }
-    ws = scratch[dev];
+    const attn_status_t s = noalloc_scratch_address(&ws);
+    if (s != ATTN_OK) return s;
   }
   return attn_decode_splitkv(q, k, v, kv_dtype, k_scale, v_scale, kv_lens, Tmax, dims, num_splits, o, lse, ws,
                              need > 0 ? (size_t)ATTN_NOALLOC_SCRATCH_BYTES : 0, stream);

@@ -40,6 +40,7 @@ struct PrefillParams {
   int n_items;       // B * n_head_units * n_q_units
   void* o;
   int o_f32;
+  long long o_sb, o_ss, o_sh;  // element strides of o between batches, tokens and heads (D contiguous)
   float* lse;
   // Packed variable-length batch (ORT packed-QSA analysis, "Code analysis": cumulative sequence
   // lengths, and a token's position = past length + its index among the new tokens): sequence b's
@@ -76,7 +77,8 @@ struct PrefillItem {
   int S, T;                    // this sequence's query and key counts
   long long q_pos0, kv_pos0;   // absolute positions of its query row 0 and key 0
   int q_base, k_base, bc;      // TMA token offsets of its rows 0 and batch coordinate
-  long long o_row0;            // row of query 0 in o / lse (rows of Hq heads)
+  long long o_base;            // element offset of query 0's row in o
+  long long lse_row0;          // row of query 0 in lse (rows of Hq heads)
 };
 
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int idx) {
@@ -96,7 +98,8 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
     it.q_base = qs;
     it.k_base = ks;
     it.bc = 0;
-    it.o_row0 = qs;
+    it.o_base = (long long)qs * p.o_ss;
+    it.lse_row0 = qs;
   } else {
     it.S = p.S;
     it.T = p.T;
@@ -105,7 +108,8 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
     it.q_base = 0;
     it.k_base = 0;
     it.bc = it.b;
-    it.o_row0 = (long long)it.b * p.S;
+    it.o_base = (long long)it.b * p.o_sb;
+    it.lse_row0 = (long long)it.b * p.S;
   }
   for (int s = 0; s < 2; ++s) {
     int head, qt;
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(384, 1)
     if (r == 0) ATTN_TRACE_AT(4 + slot, 2, ok);
     if (ok) {
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const long long orow = ((it.o_row0 + row) * p.Hq + it.head[slot]) * D;
+      const long long orow = it.o_base + (long long)row * p.o_ss + (long long)it.head[slot] * p.o_sh;
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
         if (have_o) {  // warp-collective load for every lane; only rows < S are stored
@@ -464,7 +468,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (p.lse && row_ok) {
         const float lse = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        p.lse[(it.o_row0 + row) * p.Hq + it.head[slot]] = lse;
+        p.lse[(it.lse_row0 + row) * p.Hq + it.head[slot]] = lse;
       }
     }
   }

@@ -254,7 +254,7 @@ attn_status_t attn_chunked_stream(const void* q_h, const void* k_h, const void* 
         attn_dims_t dd = d;
         const bool first = (j == 0);
         s2 = attn_prefill(qbuf[qb], kbuf[kb], vbuf[kb], first ? o_acc : o_tmp, ATTN_F32,
-                          static_cast<float*>(first ? l_acc : l_tmp), dd, (int)rows, (int)klen, causal, q0, k0, cs);
+                          static_cast<float*>(first ? l_acc : l_tmp), dd, (int)rows, (int)klen, causal, q0, k0, nullptr, cs);
         if (s2 != ATTN_OK) return s2;
         if (!first) {
           s2 = attn_merge_lse(static_cast<float*>(o_tmp), static_cast<float*>(l_tmp), 1, B * rows * d.Hq, d.D, o_acc,

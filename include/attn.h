@@ -19,7 +19,8 @@
  *   [ORT-CPU] "ONNX Runtime CPU GQA optimization: Flash Attention and Flash Decoding"
  *           (analysis of onnxruntime PR 28695), Code analysis 1-2, Reviewer feedback.
  *   [ORT-QSA] "ONNX Runtime CUDA packed sparse attention optimization" (analysis of
- *           onnxruntime PR 33328), Code analysis 1.
+ *           onnxruntime PR 33328), Code analysis 1 (packed tokens, positions) and 2 (multi-token
+ *           verification).
  *
  * Conventions for every entry point
  *   - Device pointers are plain CUDA device addresses owned by the caller; the library never
@@ -90,13 +91,25 @@ typedef struct {
  *
  *   q    device bf16 [B, S, Hq, D]     k, v  device bf16 [B, T, Hkv, D]
  *   o    device [B, S, Hq, D], bf16 (o_dtype = ATTN_BF16) or float32 (ATTN_F32)
- *   lse  device float32 [B, S, Hq] or NULL.  Rows that see no key get O = 0, LSE = -inf.
+ *   lse  device float32 [B, S, Hq] (always packed) or NULL.  Rows that see no key get O = 0,
+ *        LSE = -inf.
  *   S, T >= 0 (S = 0 or B = 0 is a no-op); q_pos0, kv_pos0 >= 0.
+ *   strides  host array of 12 element strides, or NULL for packed [B, S, H, D] tensors:
+ *        {q_b, q_s, q_h, k_b, k_s, k_h, v_b, v_s, v_h, o_b, o_s, o_h}, the distance in elements
+ *        between consecutive batches, tokens and heads of q, k, v and o; the D elements of a head
+ *        are always contiguous.  Views such as one slice of a fused [B, S, Hq + 2 Hkv, D] QKV
+ *        tensor, a subset of heads, or a [B, H, S, D] tensor seen as [B, S, H, D] are read in
+ *        place, with no copy ([ORT-QSA] Code analysis 1: Q, K and V packed in one tensor).  Each
+ *        stride must be positive and a whole number of 16-byte units (a multiple of 8 elements;
+ *        of 4 for a float32 o); the array is read during the call only.  The caller keeps the
+ *        rows o addresses disjoint.
+ * Errors: ATTN_ERR_INVALID_ARG for bad sizes, strides, null or misaligned pointers;
+ * ATTN_ERR_UNSUPPORTED for other head dims; ATTN_ERR_CUDA if the driver refuses a tensor map.
  * Returns ATTN_OK after enqueueing on `stream`.
  * ------------------------------------------------------------------------------------------ */
 ATTN_API attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* o, attn_dtype_t o_dtype,
                            float* lse, attn_dims_t dims, int S, int T, int causal, long long q_pos0,
-                           long long kv_pos0, void* stream);
+                           long long kv_pos0, const long long* strides, void* stream);
 
 /* ------------------------------------------------------------------------------------------
  * attn_prefill_varlen — attn_prefill over a packed batch of sequences of different lengths,
@@ -161,8 +174,8 @@ ATTN_API attn_status_t attn_decode_splitkv(const void* q, const void* k, const v
  * attn_decode_multi — n_q query tokens per sequence over one KV cache (multi-token decode,
  * e.g. verifying n_q draft tokens).
  *
- * [ORT-GQA] Code analysis 4 (packed QKV with past lengths): a new token's absolute position is
- * the past length plus its index among the new tokens.  Here the cache already holds the n_q
+ * [ORT-QSA] Code analysis 2 (multi-token verification; positions of packed tokens): a new
+ * token's absolute position is the past length plus its index among the new tokens.  Here the cache already holds the n_q
  * new tokens, so token i of sequence b sits at position kv_lens[b] - n_q + i and sees keys
  * [0, kv_lens[b] - n_q + i + 1) (a token with no visible key gets O = 0, LSE = -inf).  One pass
  * over the cache serves all n_q tokens: their n_q * Hq/Hkv query rows share each K/V tile, which
@@ -220,7 +233,11 @@ ATTN_API attn_status_t attn_decode_paged(const void* q, const void* k_pool, cons
  * process exits.  It allocates nothing.
  *
  *   - The first call on a device (with that device current) looks up the array's device
- *     address; make that first call before any stream capture.
+ *     address; make that first call before any stream capture.  The address is kept with the
+ *     device's context and looked up again if that context changes (e.g. after cudaDeviceReset,
+ *     which reloads the library's device code).
+ *   - The arguments are checked first, exactly as attn_decode_splitkv checks them (an invalid or
+ *     unsupported call gets that status whatever its size); the scratch limit after them.
  *   - Requests whose partials need more than ATTN_NOALLOC_SCRATCH_BYTES
  *     (attn_decode_workspace_bytes(dims, Tmax, num_splits) > the limit) return ATTN_ERR_BUDGET
  *     without launching anything; lower num_splits or use attn_decode_splitkv.
@@ -315,7 +332,7 @@ ATTN_API attn_status_t attn_set_wait_limit_ns(unsigned long long ns);
  * the timeout path without faulting or hanging the GPU.  Synchronises the device. */
 ATTN_API attn_status_t attn_debug_wait_probe(unsigned long long limit_ns);
 /* Evaluates the kernels' exp2 on n device floats: mode 0 = the FMA-pipe polynomial the prefill
- * softmax uses for a quarter of its exponentials, mode 1 = the MUFU ex2.approx.  For tests. */
+ * softmax uses for one exponential pair in eight, mode 1 = the MUFU ex2.approx.  For tests. */
 ATTN_API attn_status_t attn_debug_exp2(const float* x, float* y, long long n, int mode, void* stream);
 /* Host-side fault injection for the streamer: the nth (1-based) host->device copy (what = 1)
  * or device allocation (what = 2) of the next attn_chunked_stream call fails with

@@ -105,8 +105,10 @@ def decode(q, k, v, kv_lens, *, scale: float, k_scale=None, v_scale=None):
 
 def decode_multi(q, k, v, kv_lens, *, scale: float, k_scale=None, v_scale=None):
     """Multi-token decode: the cache already holds the n_q new tokens, so token i of sequence b
-    is at position len_b - n_q + i (past length + index among the new tokens, as the ORT GQA
-    analysis positions packed tokens, "Code analysis 4") and attends causally to the cache.
+    is at position len_b - n_q + i (past length + index among the new tokens, as the ORT CUDA
+    packed sparse attention analysis positions packed tokens in "Code analysis" 1 and verifies
+    several new tokens against one key state in "Code analysis" 2) and attends causally to the
+    cache.
 
     q: [B, n_q, Hq, D]; k, v: [B, Tmax, Hkv, D]; kv_lens [B].
     Returns (o [B, n_q, Hq, D], lse [B, n_q, Hq]).

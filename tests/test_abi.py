@@ -62,18 +62,44 @@ def test_prefill_invalid_args(L, case):
              q_pos0=0, kv_pos0=0)
     a.update(case)
     st = L.attn_prefill(a["q"], a["k"], a["v"], a["o"], a["o_dtype"], a["lse"], a["dims"], a["S"], a["T"],
-                        a["causal"], a["q_pos0"], a["kv_pos0"], None)
+                        a["causal"], a["q_pos0"], a["kv_pos0"], a.get("strides"), None)
     assert st == 1
 
 
 def test_prefill_unsupported_head_dim(L):
-    st = L.attn_prefill(FAKE, FAKE, FAKE, FAKE, 0, None, _dims(D=96), 16, 16, 1, 0, 0, None)
+    st = L.attn_prefill(FAKE, FAKE, FAKE, FAKE, 0, None, _dims(D=96), 16, 16, 1, 0, 0, None, None)
     assert st == 2
 
 
 def test_prefill_empty_is_noop(L):
-    assert L.attn_prefill(None, None, None, None, 0, None, _dims(B=0), 16, 16, 1, 0, 0, None) == 0
-    assert L.attn_prefill(None, None, None, None, 0, None, _dims(), 0, 16, 1, 0, 0, None) == 0
+    assert L.attn_prefill(None, None, None, None, 0, None, _dims(B=0), 16, 16, 1, 0, 0, None, None) == 0
+    assert L.attn_prefill(None, None, None, None, 0, None, _dims(), 0, 16, 1, 0, 0, None, None) == 0
+
+
+def _strides(**bad):
+    """Packed [B=1, S=16, H, D=64] strides for q/o (Hq=4) and k/v (Hkv=2), with overrides."""
+    base = dict(q_b=16 * 4 * 64, q_s=4 * 64, q_h=64, k_b=16 * 2 * 64, k_s=2 * 64, k_h=64,
+                v_b=16 * 2 * 64, v_s=2 * 64, v_h=64, o_b=16 * 4 * 64, o_s=4 * 64, o_h=64)
+    base.update(bad)
+    order = ["q_b", "q_s", "q_h", "k_b", "k_s", "k_h", "v_b", "v_s", "v_h", "o_b", "o_s", "o_h"]
+    return (ctypes.c_longlong * 12)(*[base[n] for n in order])
+
+
+@pytest.mark.parametrize("bad", [dict(q_h=0), dict(k_s=-128), dict(v_b=4), dict(o_h=68), dict(q_s=1 << 40),
+                                 dict(k_h=63)])
+def test_prefill_invalid_strides(L, bad):
+    """Each stride must be positive, a whole number of 16-byte units and below TMA's limit; the
+    check runs before any CUDA call (the pointers here are never dereferenced)."""
+    st = L.attn_prefill(FAKE, FAKE, FAKE, FAKE, 0, None, _dims(), 16, 16, 1, 0, 0, _strides(**bad), None)
+    assert st == 1
+
+
+def test_prefill_float32_output_strides_in_4_element_units(L):
+    """A float32 o needs its strides in 16-byte units = 4 elements; 68 is one, not for bf16."""
+    st = L.attn_prefill(FAKE, FAKE, FAKE, FAKE, 2, None, _dims(D=96), 16, 16, 1, 0, 0, _strides(o_h=68), None)
+    assert st == 2  # strides accepted; the head dim is what is unsupported
+    st = L.attn_prefill(FAKE, FAKE, FAKE, FAKE, 0, None, _dims(D=96), 16, 16, 1, 0, 0, _strides(o_h=68), None)
+    assert st == 1
 
 
 @pytest.mark.parametrize("case", [

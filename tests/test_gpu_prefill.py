@@ -94,3 +94,72 @@ def test_prefill_b2_h32_d128_s8192_sampled(cuda_device):
     q, k, v = I.prefill_inputs(w)
     rows = I.sample_rows(w.S, 48, seed=77, edges=(0, 1, 127, 128, 4095, 4096, 8191))
     _check(q, k, v, cuda_device, causal=True, rows=rows)
+
+
+def _check_views(qv, kv, vv, dev, causal=True, o=None, scale=None):
+    """attn_prefill on strided views (read in place through the strides argument) against the
+    oracle on packed copies of the same values."""
+    D = qv.shape[-1]
+    scale = 1 / math.sqrt(D) if scale is None else scale
+    o, lse = A.attn_prefill(qv, kv, vv, causal=causal, o=o, scale=scale)
+    torch.cuda.synchronize()
+    ro, rl = O.attention(qv.cpu().contiguous(), kv.cpu().contiguous(), vv.cpu().contiguous(), scale=scale,
+                         causal=causal)
+    assert_o_close(o, ro)
+    assert_lse_close(to_np(lse).transpose(0, 2, 1), rl)
+    device_clean()
+    return o
+
+
+def test_prefill_fused_qkv_views(cuda_device):
+    """Q, K and V as slices of one fused [B, S, Hq + 2 Hkv, D] tensor (packed QKV), ragged length."""
+    B, S, Hq, Hkv, D = 2, 300, 8, 2, 128
+    g = I.generator(21)
+    qkv = I.randn_bf16((B, S, Hq + 2 * Hkv, D), g).to(cuda_device)
+    q, k, v = qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:]
+    assert not q.is_contiguous() and not k.is_contiguous()
+    _check_views(q, k, v, cuda_device)
+
+
+def test_prefill_head_subset_and_bhsd_views(cuda_device):
+    """Every other head of a wider tensor (head stride 2D), and K/V stored [B, H, T, D] and seen as
+    [B, T, H, D] (token stride D, head stride T*D); D = 64, non-causal, 5 key tiles."""
+    B, S, T, Hq, Hkv, D = 1, 200, 600, 4, 2, 64
+    g = I.generator(22)
+    qw = I.randn_bf16((B, S, 2 * Hq, D), g).to(cuda_device)
+    k_bhsd = I.randn_bf16((B, Hkv, T, D), g).to(cuda_device)
+    v_bhsd = I.randn_bf16((B, Hkv, T, D), g).to(cuda_device)
+    q = qw[:, :, ::2]
+    k, v = k_bhsd.transpose(1, 2), v_bhsd.transpose(1, 2)
+    _check_views(q, k, v, cuda_device, causal=False)
+
+
+def test_prefill_strided_output_leaves_neighbours(cuda_device):
+    """O written into a head slice of a wider buffer (bf16 and float32): the slice matches the
+    oracle and the heads around it keep their sentinel values."""
+    B, S, Hq, Hkv, D = 1, 257, 4, 2, 128
+    q, k, v = _gen(B, S, S, Hq, Hkv, D, seed=23)
+    for dt in (torch.bfloat16, torch.float32):
+        wide = torch.full((B, S, Hq + 3, D), 7.0, dtype=dt, device=cuda_device)
+        o = wide[:, :, 1:1 + Hq]
+        _check_views(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), cuda_device, o=o)
+        assert torch.all(wide[:, :, 0] == 7.0) and torch.all(wide[:, :, 1 + Hq:] == 7.0)
+
+
+def test_prefill_strided_no_visible_keys(cuda_device):
+    """A strided call with no keys, and one whose first query tile sees none (key chunk after the
+    queries): empty rows get O = 0 and LSE = -inf from the kernel itself."""
+    B, S, Hq, Hkv, D = 1, 300, 4, 2, 128
+    g = I.generator(24)
+    qkv = I.randn_bf16((B, S, Hq + 2 * Hkv, D), g).to(cuda_device)
+    q, k, v = qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:]
+    o, lse = A.attn_prefill(q, k[:, :0], v[:, :0], causal=True)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+    o, lse = A.attn_prefill(q, k, v, causal=True, q_pos0=0, kv_pos0=200)
+    torch.cuda.synchronize()
+    ro, rl = O.attention(q.cpu().contiguous(), k.cpu().contiguous(), v.cpu().contiguous(), scale=1 / math.sqrt(D),
+                         causal=True, q_pos0=0, kv_pos0=200)
+    assert_o_close(o, ro)
+    assert_lse_close(to_np(lse).transpose(0, 2, 1), rl)
+    device_clean()

@@ -5,8 +5,9 @@ nearly all of the GPU's memory for its own pool, or a latency-critical decode lo
 a cudaMalloc (which may synchronise the device) is not allowed.  For them the library keeps
 the split-KV partials in one static device array instead of a caller-provided workspace.
 These tests call that entry point through the C ABI and check that it gives the same result
-as attn_decode_splitkv with a workspace, on two calls in a row (the array keeps the previous
-call's contents, which must not leak into the next result), and that it allocates nothing.
+as attn_decode_splitkv with a workspace and as the float64 oracle, on two calls in a row (the
+array keeps the previous call's contents, which must not leak into the next result), and that
+it allocates nothing; one more call goes through the Python wrapper with preallocated outputs.
 This file is collected last on purpose.
 """
 import ctypes
@@ -18,7 +19,9 @@ import torch
 
 from exact_long_context_tmem_b200 import attn as A
 from exact_long_context_tmem_b200 import inputs as I
-from tests.parity import LSE_ATOL, O_ATOL, O_RTOL
+from oracle import attention as OR
+from oracle import fp8 as F8
+from tests.parity import LSE_ATOL, O_ATOL, O_RTOL, assert_lse_close, assert_o_close
 
 LIMIT = 4 << 20  # ATTN_NOALLOC_SCRATCH_BYTES in include/attn.h
 
@@ -70,13 +73,30 @@ def test_noalloc_matches_workspace_decode_two_calls(cuda_device):
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     assert free1 == free0, "the no-allocation entry point changed device memory use"
-    for w, dd, splits, ref_o, ref_l, o, lse in outs:
+    for ((w, d), _), (w2, dd, splits, ref_o, ref_l, o, lse) in zip(cases, outs):
         ro, go = ref_o.float().cpu().numpy(), o.float().cpu().numpy()
         assert np.all(np.abs(go - ro) <= O_ATOL + O_RTOL * np.abs(ro))
         rl, gl = ref_l.cpu().numpy(), lse.cpu().numpy()
         np.testing.assert_array_equal(np.isneginf(gl), np.isneginf(rl))
         fin = np.isfinite(rl)
         assert np.all(np.abs(gl[fin] - rl[fin]) <= LSE_ATOL)
+        # and against the float64 oracle on the same seeded inputs
+        if "k_codes" in d:
+            kv, vv = F8.e4m3_decode(d["k_codes"]), F8.e4m3_decode(d["v_codes"])
+            oo, ol = OR.decode(d["q"], kv, vv, d["kv_lens"], scale=w.scale, k_scale=d["k_scale"],
+                               v_scale=d["v_scale"])
+        else:
+            oo, ol = OR.decode(d["q"], d["k"], d["v"], d["kv_lens"], scale=w.scale)
+        assert_o_close(o, oo, "no-alloc O vs oracle")
+        assert_lse_close(lse, ol, "no-alloc LSE vs oracle")
+    # one more call through the Python wrapper, into preallocated outputs
+    w, dd, splits, ref_o, ref_l, o, lse = outs[0]
+    o.fill_(float("nan"))
+    lse.fill_(float("nan"))
+    A.attn_decode_splitkv_noalloc(dd["q"], dd["k"], dd["v"], dd["kv_lens"], num_splits=splits, o=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) or np.all(np.abs(o.float().cpu().numpy() - ref_o.float().cpu().numpy())
+                                          <= O_ATOL + O_RTOL * np.abs(ref_o.float().cpu().numpy()))
     st, site = A.attn_device_status(reset=True)
     assert st == 0, f"device status {st} at wait site {site}"
 
@@ -92,3 +112,17 @@ def test_noalloc_rejects_requests_beyond_the_scratch_limit():
     st = L.attn_decode_splitkv_noalloc(fake, fake, fake, A.ATTN_BF16, None, None, fake, 131072, dims, 1024, fake,
                                        None, None)
     assert st == 4  # ATTN_ERR_BUDGET
+
+
+@pytest.mark.parametrize("bad,status", [("q", 1), ("head_dim", 2)])
+def test_noalloc_argument_errors_come_before_the_limit(bad, status):
+    """A request beyond the scratch limit that is also malformed (a null query) or unsupported
+    (head dim 96) reports that, not the limit: the checks run in attn_decode_splitkv's order
+    first (no GPU needed: nothing is launched)."""
+    L = A.lib()
+    dims = A.Dims(64, 32, 8, 96 if bad == "head_dim" else 128, 0.088)
+    fake = ctypes.c_void_p(0x10000)
+    q = None if bad == "q" else fake
+    st = L.attn_decode_splitkv_noalloc(q, fake, fake, A.ATTN_BF16, None, None, fake, 131072, dims, 1024, fake,
+                                       None, None)
+    assert st == status
