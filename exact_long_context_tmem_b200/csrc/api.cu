@@ -107,6 +107,21 @@ static constexpr float kLog2e = 1.4426950408889634f;
 // cut by the device cumulative lengths, and max_s the longest query count (grid size).
 // strides: NULL (packed [B, S, H, D] tensors) or 12 element strides, (batch, token, head) for
 // q, k, v and o in that order; already validated.
+// A kernel whose warpgroups trade registers with setmaxnreg must be launched with at least the
+// registers the split hands out, or the increasing warpgroups wait forever: check the compiled
+// per-thread count once (per kernel) before the first launch.
+template <typename K>
+static attn_status_t check_register_split(K kernel, int threads, int split_total, std::atomic<int>& state) {
+  int s = state.load(std::memory_order_acquire);
+  if (s == 0) {
+    cudaFuncAttributes a{};
+    ATTN_CUDA(cudaFuncGetAttributes(&a, kernel));
+    s = (a.numRegs * threads >= split_total) ? 1 : 2;
+    state.store(s, std::memory_order_release);
+  }
+  return s == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+}
+
 template <int D>
 static attn_status_t launch_prefill(const void* q, const void* k, const void* v, void* o, int o_f32, float* lse,
                                     const attn_dims_t& d, int S, int T, int causal, long long q_pos0,
@@ -114,7 +129,11 @@ static attn_status_t launch_prefill(const void* q, const void* k, const void* v,
                                     const int* cu_k = nullptr, int max_s = 0, const long long* strides = nullptr) {
   using C = PrefillCfg<D>;
   static std::atomic<uint64_t> smem_done{0};
+  static std::atomic<int> regs_state{0};
   attn_status_t st = ensure_smem(prefill_fwd_sm100<D>, C::SMEM_BYTES, smem_done);
+  if (st != ATTN_OK) return st;
+  st = check_register_split(prefill_fwd_sm100<D>, C::THREADS, C::REGS_CTRL * 128 + C::REGS_SOFTMAX * 256,
+                            regs_state);
   if (st != ATTN_OK) return st;
   CUtensorMap mq, mk, mv;
   const uint64_t nb = cu_q ? 1 : (uint64_t)d.B;

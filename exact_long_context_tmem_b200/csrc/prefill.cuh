@@ -5,7 +5,7 @@
 // compute the score block, update the running row max and row sum (online softmax), and
 // accumulate P.V into the output; the S x T score matrix never leaves the SM.
 //
-// Roles (384 threads):
+// Roles (384 threads; warpgroup 0 hands most of its registers to warpgroups 1 and 2):
 //   warp 0        TMA producer: Q tiles once, then K_j / V_j through an NST-stage ring
 //   warp 1        TMEM allocator; lane 0 issues every tcgen05.mma and commit
 //   warps 4..7    softmax + epilogue for slot 0 (one thread per TMEM lane = query row)
@@ -18,15 +18,15 @@
 
 #include "ptx.cuh"
 
-// One in this many exponential pairs of the softmax is computed by polynomial on the FMA pipe
-// instead of the MUFU (0: all on the MUFU).
-#ifndef ATTN_PREFILL_POLY_PERIOD
-#define ATTN_PREFILL_POLY_PERIOD 8
+// Of every 8 exponential pairs of the softmax, this many are computed by polynomial on the FMA
+// pipe instead of the MUFU (0: all on the MUFU).
+#ifndef ATTN_PREFILL_POLY_PER8
+#define ATTN_PREFILL_POLY_PER8 1
 #endif
 
 namespace attn {
 
-constexpr int kPolyPeriod = ATTN_PREFILL_POLY_PERIOD;
+constexpr int kPolyPer8 = ATTN_PREFILL_POLY_PER8;
 
 struct PrefillParams {
   int B, Hq, Hkv, D, S, T, G;
@@ -65,6 +65,11 @@ struct PrefillCfg {
   static constexpr int N_BARS = 1 + 4 * NST + 2 + 2 + 1 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
+  // Register split (setmaxnreg): the producer / MMA warpgroup gives registers to the two softmax
+  // warpgroups, which hold a row's 128 scores and weights.  REGS_CTRL * 128 + REGS_SOFTMAX * 256
+  // must not exceed the launch allocation (the host checks it against the compiled count).
+  static constexpr int REGS_CTRL = 72;
+  static constexpr int REGS_SOFTMAX = 216;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when max grows > 2^8
 };
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 4);  // one arrival per softmax warp
     }
     mbar_init(o_full, 1);
     mbar_init(drain, 1);
@@ -197,16 +202,21 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
+    regs_dec<C::REGS_CTRL>();
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      // L2: a Q tile is read once (evict first); a K/V tile is read by every query tile of its
+      // head group, so it is kept (evict last) against the streamed Q reads and O writes.
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
       uint8_t* sQ = smem + C::OFF_Q;
       mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
       for (int s = 0; s < 2; ++s)
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(sQ + s * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, q_full, bx * 64, it.head[s],
-                      it.q_base + it.q_lo[s], it.bc);
+          tma_load_4d_hint(sQ + s * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, q_full, bx * 64, it.head[s],
+                           it.q_base + it.q_lo[s], it.bc, pol_q);
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < n && ok; ++j) {
@@ -216,14 +226,14 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&k_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; break; }
         mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem + C::OFF_K + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmK, &k_full[st], bx * 64, it.kvh,
-                      it.k_base + j * 128, it.bc);
+          tma_load_4d_hint(smem + C::OFF_K + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmK, &k_full[st], bx * 64,
+                           it.kvh, it.k_base + j * 128, it.bc, pol_kv);
         ATTN_TRACE_AT(0, 5, j);
         if (!mbar_wait(&v_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; issued = 2 * j + 1; break; }
         mbar_arrive_expect_tx(&v_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem + C::OFF_V + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmV, &v_full[st], bx * 64, it.kvh,
-                      it.k_base + j * 128, it.bc);
+          tma_load_4d_hint(smem + C::OFF_V + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmV, &v_full[st], bx * 64,
+                           it.kvh, it.k_base + j * 128, it.bc, pol_kv);
         issued = 2 * j + 2;
       }
       ATTN_TRACE_AT(0, 6, issued);
@@ -240,42 +250,50 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop in lockstep and one elected lane issues each MMA and commit:
+    // descriptors are base values computed once plus compile-time offsets of their start-address
+    // field (addresses stay below 2^18 bytes, so the field never carries), so an MMA costs the
+    // issuing warp a couple of uniform instructions even while the softmax warps sharing its
+    // sub-partition keep the issue slots busy.
+    regs_dec<C::REGS_CTRL>();
+    {
       constexpr uint32_t idesc_qk = make_idesc_f16(128, 128, false, false, true);
       constexpr uint32_t idesc_pv = make_idesc_f16(128, D, false, true, true);
-      const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-      const uint32_t sK = smem_u32(smem + C::OFF_K);
-      const uint32_t sV = smem_u32(smem + C::OFF_V);
-      const uint32_t tS[2] = {tmem + 0, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      constexpr uint32_t HI = sdesc_sw128_hi(1024);  // every operand here: 8-row groups 1024 B apart
+      const uint32_t q_lo = sdesc_sw128_lo(smem_u32(smem + C::OFF_Q), 16);
+      const uint32_t k_lo = sdesc_sw128_lo(smem_u32(smem + C::OFF_K), 16);
+      const uint32_t v_lo = sdesc_sw128_lo(smem_u32(smem + C::OFF_V), C::BOX_BYTES);
       auto issue_qk = [&](int s, int st) {
+        const uint32_t a0 = q_lo + ((s * C::TILE_BYTES) >> 4), b0 = k_lo + ((st * C::TILE_BYTES) >> 4);
+        const uint32_t d = tmem + s * 128;
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          const uint64_t da = make_sdesc_sw128(sQ + s * C::TILE_BYTES + off, 16, 1024);
-          const uint64_t db = make_sdesc_sw128(sK + st * C::TILE_BYTES + off, 16, 1024);
-          mma_ss(tS[s], da, db, idesc_qk, kk > 0);
+          const uint32_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+          mma_ss_elect(d, sdesc_join(a0 + off, HI), sdesc_join(b0 + off, HI), idesc_qk, kk > 0);
         }
       };
       auto issue_pv = [&](int s, int st, bool acc) {
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint64_t db = make_sdesc_sw128(sV + st * C::TILE_BYTES + kk * 16 * 128, C::BOX_BYTES, 1024);
-          mma_ts(tO[s], tS[s] + kk * 8, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
+        const uint32_t b0 = v_lo + ((st * C::TILE_BYTES) >> 4);
+        const uint32_t d = tmem + 256 + s * D, a = tmem + s * 128;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts_elect(d, a + kk * 8, sdesc_join(b0 + ((kk * 16 * 128) >> 4), HI), idesc_pv,
+                       (acc || kk > 0) ? 1u : 0u);
       };
-      ATTN_TRACE_AT(1, 3, 0);
-      bool ok = mbar_wait(q_full, 0, SITE_PF_MMA_Q);
-      ATTN_TRACE_AT(1, 4, ok);
+      if (lane == 0) ATTN_TRACE_AT(1, 3, 0);
+      bool ok = mbar_wait_warp(q_full, 0, SITE_PF_MMA_Q);
+      if (lane == 0) ATTN_TRACE_AT(1, 4, ok);
       if (ok && n > 0) {
-        ok = mbar_wait(&k_full[0], 0, SITE_PF_MMA_K);
+        ok = mbar_wait_warp(&k_full[0], 0, SITE_PF_MMA_K);
         if (ok) {
           tc_fence_after();
-          ATTN_EVT(0, 0);
+          if (lane == 0) ATTN_EVT(0, 0);
           issue_qk(0, 0);
-          mma_commit(&s_full[0]);
-          ATTN_EVT(0, 8);
+          mma_commit_elect(&s_full[0]);
+          if (lane == 0) ATTN_EVT(0, 8);
           issue_qk(1, 0);
-          mma_commit(&s_full[1]);
-          mma_commit(&k_empty[0]);
+          mma_commit_elect(&s_full[1]);
+          mma_commit_elect(&k_empty[0]);
         }
       }
       for (int j = 0; j < n && ok; ++j) {
@@ -284,45 +302,48 @@ __global__ void __launch_bounds__(384, 1)
         const bool more = j + 1 < n;
         const int st1 = (j + 1) % C::NST;
         const uint32_t ph1 = ((j + 1) / C::NST) & 1;
-        ATTN_TRACE_AT(1, 5, j);
-        if (!(ok = mbar_wait(&v_full[st], ph, SITE_PF_MMA_V))) break;
-        ATTN_TRACE_AT(1, 6, j);
-        if (!(ok = mbar_wait(&p_full[0], j & 1, SITE_PF_MMA_P))) break;
-        ATTN_TRACE_AT(1, 7, j);
+        if (lane == 0) ATTN_TRACE_AT(1, 5, j);
+        if (!(ok = mbar_wait_warp(&v_full[st], ph, SITE_PF_MMA_V))) break;
+        if (lane == 0) ATTN_TRACE_AT(1, 6, j);
+        if (!(ok = mbar_wait_warp(&p_full[0], j & 1, SITE_PF_MMA_P))) break;
+        if (lane == 0) ATTN_TRACE_AT(1, 7, j);
         tc_fence_after();
-        ATTN_EVT(j, 3);
+        if (lane == 0) ATTN_EVT(j, 3);
         issue_pv(0, st, j > 0);
         if (more) {
-          if (!(ok = mbar_wait(&k_full[st1], ph1, SITE_PF_MMA_K))) break;
+          if (!(ok = mbar_wait_warp(&k_full[st1], ph1, SITE_PF_MMA_K))) break;
           tc_fence_after();
-          ATTN_EVT(j + 1, 0);
+          if (lane == 0) ATTN_EVT(j + 1, 0);
           issue_qk(0, st1);
-          mma_commit(&s_full[0]);
+          mma_commit_elect(&s_full[0]);
         }
-        ATTN_TRACE_AT(1, 8, j);
-        if (!(ok = mbar_wait(&p_full[1], j & 1, SITE_PF_MMA_P))) break;
-        ATTN_TRACE_AT(1, 9, j);
+        if (lane == 0) ATTN_TRACE_AT(1, 8, j);
+        if (!(ok = mbar_wait_warp(&p_full[1], j & 1, SITE_PF_MMA_P))) break;
+        if (lane == 0) ATTN_TRACE_AT(1, 9, j);
         tc_fence_after();
-        ATTN_EVT(j, 11);
+        if (lane == 0) ATTN_EVT(j, 11);
         issue_pv(1, st, j > 0);
-        mma_commit(&v_empty[st]);
+        mma_commit_elect(&v_empty[st]);
         if (more) {
-          ATTN_EVT(j + 1, 8);
+          if (lane == 0) ATTN_EVT(j + 1, 8);
           issue_qk(1, st1);
-          mma_commit(&s_full[1]);
-          mma_commit(&k_empty[st1]);
+          mma_commit_elect(&s_full[1]);
+          mma_commit_elect(&k_empty[st1]);
         }
       }
-      if (ok && n > 0) mma_commit(o_full);
-      ATTN_TRACE_AT(1, 10, ok);
+      if (ok && n > 0) mma_commit_elect(o_full);
+      if (lane == 0) ATTN_TRACE_AT(1, 10, ok);
       // Drain: every MMA issued above completes before TMEM is released.
-      mma_commit(drain);
+      mma_commit_elect(drain);
       const bool drained = mbar_wait_drain(drain, 0, SITE_PF_DRAIN);
-      ATTN_TRACE_AT(1, 11, drained);
+      if (lane == 0) ATTN_TRACE_AT(1, 11, drained);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    regs_dec<C::REGS_CTRL>();  // idle warps of warpgroup 0: give their registers away
+  } else {
     // ------------------------------------------------------------------ softmax + epilogue
+    regs_inc<C::REGS_SOFTMAX>();
     const int slot = (warp - 4) >> 2;
     const int wq = warp & 3;  // TMEM lane quarter this warp may access
     const int r = wq * 32 + lane;
@@ -390,12 +411,12 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (r == 0) ATTN_EVT(j, slot * 8 + 2);
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      // p = 2^(s * scale * log2 e - m) in packed fp32 pairs; one pair in ATTN_PREFILL_POLY_PERIOD
-      // goes to the FMA pipe (polynomial) and the rest to the MUFU.  P is stored per 32 scores (16 packed columns, over
-      // S columns already read into registers) so those registers retire early.
+      // p = 2^(s * scale * log2 e - m) in packed fp32 pairs; ATTN_PREFILL_POLY_PER8 pairs in 8 go
+      // to the FMA pipe (polynomial) and the rest to the MUFU.  P is stored per 32 scores (16
+      // packed columns, over S columns already read into registers).  The fp32 weights stay in the
+      // score registers: the row sum is taken after P is handed to the MMA, off the critical path.
       const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nm2 = make_float2(neg_m, neg_m);
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -404,25 +425,40 @@ __global__ void __launch_bounds__(384, 1)
           const int k = c * 32 + 2 * i;
           const float2 x = fma2(make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), c2, nm2);
           float2 e;
-          if (kPolyPeriod > 0 && i % (kPolyPeriod > 0 ? kPolyPeriod : 1) == kPolyPeriod - 1) {
+          if ((i & 7) >= 8 - kPolyPer8) {
             e = exp2_poly2(x);
           } else {
             e.x = ex2_approx(x.x);
             e.y = ex2_approx(x.y);
           }
           pk[i] = pack_bf16x2(e.x, e.y);
-          if (i & 1) acc1 = add2(acc1, e);
-          else acc0 = add2(acc0, e);
+          sr[k] = __float_as_uint(e.x);
+          sr[k + 1] = __float_as_uint(e.y);
         }
         tmem_st16(tS + c * 16, pk);
+        if (c == 1 && r == 0) ATTN_EVT(j, slot * 8 + 6);
       }
-      l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
       if (r == 0) ATTN_TRACE_AT(2 + slot, 3, j);
       tmem_wait_st();
+      if (r == 0) ATTN_EVT(j, slot * 8 + 7);
       if (r == 0) ATTN_TRACE_AT(2 + slot, 4, j);
       tc_fence_before();
-      mbar_arrive(&p_full[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[slot]);  // one arrival per warp
       if (r == 0) ATTN_EVT(j, slot * 8 + 4);
+      {
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+#pragma unroll
+        for (int k = 0; k < 128; k += 8) {
+          a0 = add2(a0, make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])));
+          a1 = add2(a1, make_float2(__uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3])));
+          a2 = add2(a2, make_float2(__uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5])));
+          a3 = add2(a3, make_float2(__uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7])));
+        }
+        a0 = add2(add2(a0, a1), add2(a2, a3));
+        l += a0.x + a0.y;
+      }
+      if (r == 0) ATTN_EVT(j, slot * 8 + 5);
     }
     // ---- epilogue: O / l -> global, LSE = ln2 * (m + log2 l)
     const int row = q_lo + r;
@@ -451,8 +487,9 @@ __global__ void __launch_bounds__(384, 1)
           float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + orow + c * 32);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]) * inv_l, __uint_as_float(v[4 * i + 1]) * inv_l,
-                                 __uint_as_float(v[4 * i + 2]) * inv_l, __uint_as_float(v[4 * i + 3]) * inv_l);
+            st_global_cs_v4f(dst + i, make_float4(__uint_as_float(v[4 * i]) * inv_l, __uint_as_float(v[4 * i + 1]) * inv_l,
+                                                  __uint_as_float(v[4 * i + 2]) * inv_l,
+                                                  __uint_as_float(v[4 * i + 3]) * inv_l));
         } else {
           uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) + orow + c * 32);
 #pragma unroll
@@ -462,7 +499,7 @@ __global__ void __launch_bounds__(384, 1)
             w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l, __uint_as_float(v[8 * i + 3]) * inv_l);
             w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l, __uint_as_float(v[8 * i + 5]) * inv_l);
             w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l, __uint_as_float(v[8 * i + 7]) * inv_l);
-            dst[i] = w;
+            st_global_cs_v4(dst + i, w);
           }
         }
       }

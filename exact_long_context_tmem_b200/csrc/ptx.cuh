@@ -71,8 +71,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // past the deadline the wait records ATTN_ERR_TIMEOUT with a site code in the
 // device status word and returns false, and the caller unwinds.
 // A drain wait (for copies or MMAs this thread already issued, which complete on their own)
-// ignores errors recorded by other roles and only stops at the time limit.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int site, bool drain) {
+// ignores errors recorded by other roles and only stops at the time limit.  Inlined: a call
+// across warpgroups that trade registers (setmaxnreg) cannot be register-allocated.
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int site, bool drain) {
   const uint64_t t0 = globaltimer_ns();
   const uint64_t limit = g_wait_limit_ns;
   for (uint32_t it = 0;; ++it) {
@@ -151,6 +152,16 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
+// 16-byte global store that streams past the caches (evict-first: written once, read by no one here).
+__device__ __forceinline__ void st_global_cs_v4(void* dst, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_global_cs_v4f(void* dst, float4 v) {
+  asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared that reads src_bytes (0 or 16) and zero-fills the rest.
 __device__ __forceinline__ void cp_async_16_zfill(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
@@ -221,6 +232,38 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same MMAs issued by one elected lane of a converged warp: every lane passes the same
+// (warp-uniform) operands, so their arithmetic stays on the uniform datapath and the issuing warp
+// spends a few instructions per MMA.
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// tcgen05.commit from one elected lane of a converged warp.
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 
@@ -332,6 +375,19 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
   return d;
 }
 
+// The two halves of make_sdesc_sw128's result: the low word holds the start address and the
+// leading byte offset, the high word the stride byte offset, version and layout.  Descriptors that
+// share a stride share the high word, so an MMA loop can carry 32-bit low words only.
+__host__ __device__ constexpr uint32_t sdesc_sw128_hi(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t sdesc_sw128_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t sdesc_join(uint32_t lo, uint32_t hi) {
+  return ((uint64_t)hi << 32) | lo;
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128B-swizzled tile whose
 // base is 1024-byte aligned (rows are 128 bytes).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
@@ -380,11 +436,12 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // 2^x for two values on the FMA pipe instead of the MUFU: x = j + f with j = rint(x) and
-// f in [-0.5, 0.5]; 2^f by a degree-5 polynomial fitted here for minimum relative error on that
-// interval (max relative error 1.7e-7 when evaluated in float32, the accuracy class of
-// ex2.approx); 2^j is added to the
-// exponent field as an integer.  x is clamped at -127, where the construction yields exactly
-// +0.0, so masked scores (-inf) give 0 as the hardware ex2 does.
+// f in [-0.5, 0.5]; 2^f by a degree-3 polynomial with constant term 1, fitted here for minimum
+// relative error on that interval (max relative error 1.02e-4 evaluated in float32: ample for a
+// softmax weight that is rounded to bf16, 2^-9 relative, before its product with V, and a row sum
+// whose logarithm is needed to 1e-3); 2^j is added to the exponent field as an integer.  x is
+// clamped at -127, where the construction yields exactly +0.0, so masked scores (-inf) give 0 as
+// the hardware ex2 does.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer in the low bits
   x.x = fmaxf(x.x, -127.0f);
@@ -392,11 +449,9 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 t = add2(x, make_float2(kRound, kRound));
   const float2 j = add2(t, make_float2(-kRound, -kRound));
   const float2 f = add2(x, make_float2(-j.x, -j.y));
-  float2 q = fma2(make_float2(1.3264722656458616e-3f, 1.3264722656458616e-3f), f,
-                  make_float2(9.671512991189957e-3f, 9.671512991189957e-3f));
-  q = fma2(q, f, make_float2(5.550733581185341e-2f, 5.550733581185341e-2f));
-  q = fma2(q, f, make_float2(2.4022242426872253e-1f, 2.4022242426872253e-1f));
-  q = fma2(q, f, make_float2(6.931470036506653e-1f, 6.931470036506653e-1f));
+  float2 q = fma2(make_float2(5.500880256295204e-2f, 5.500880256295204e-2f), f,
+                  make_float2(2.4221086502075195e-1f, 2.4221086502075195e-1f));
+  q = fma2(q, f, make_float2(6.932829022407532e-1f, 6.932829022407532e-1f));
   q = fma2(q, f, make_float2(1.0f, 1.0f));
   const uint32_t rx = __float_as_uint(q.x) + (__float_as_uint(t.x) << 23);
   const uint32_t ry = __float_as_uint(q.y) + (__float_as_uint(t.y) << 23);

@@ -21,19 +21,20 @@ def test_wait_probe_times_out_and_context_survives(cuda_device):
 
 
 def test_polynomial_exp2_matches_float64(cuda_device):
-    """The FMA-pipe exp2 the prefill softmax uses for a quarter of its exponentials: relative
-    error within 2e-7 of float64 exp2 on the softmax's input range (x <= 8), exact 0 at and
-    below -127 (masked scores), and no worse than the MUFU ex2.approx it replaces."""
+    """The FMA-pipe exp2 the prefill softmax uses for one exponential pair in eight: relative error
+    within its fitted bound (1.02e-4, checked at 1.1e-4) of float64 exp2 on the softmax's input
+    range (x <= 8, the lazy-rescale headroom), exactly 1 at x = 0 and at the integers, and exact 0 at
+    and below -127 (masked scores).  The bound is far inside what a weight rounded to bf16 (2^-9)
+    and a row sum needed to 1e-3 in log space can tell apart."""
     import numpy as np
     g = torch.Generator().manual_seed(3)
     x = torch.cat([torch.linspace(-126.0, 8.0, 2_000_001), torch.rand(1_000_000, generator=g) * 28 - 20,
                    torch.tensor([0.0, 0.5, -0.5, 8.0, -1e-30, 1e-30])]).float()
     ref = np.exp2(x.double().numpy())
     y_poly = A.attn_debug_exp2(x.to(cuda_device), mode=0).cpu().double().numpy()
-    y_mufu = A.attn_debug_exp2(x.to(cuda_device), mode=1).cpu().double().numpy()
     rel_poly = np.abs(y_poly / ref - 1)
-    rel_mufu = np.abs(y_mufu / ref - 1)
-    assert rel_poly.max() <= 2e-7, rel_poly.max()
-    assert rel_poly.max() <= 2 * rel_mufu.max() + 1e-7
+    assert rel_poly.max() <= 1.1e-4, rel_poly.max()
+    ints = torch.arange(-126, 9, dtype=torch.float32)
+    assert torch.equal(A.attn_debug_exp2(ints.to(cuda_device), mode=0).cpu(), torch.exp2(ints))
     z = torch.tensor([-float("inf"), -1000.0, -200.0, -127.0], device=cuda_device)
     assert torch.all(A.attn_debug_exp2(z, mode=0) == 0)
