@@ -2,13 +2,14 @@
 """Benchmark of the exact-attention hot path on B200.
 
 Headline: causal GQA prefill, batch 2, 32 query / 8 KV heads, head dim 128, 8192 tokens,
-bf16 in / fp32 accumulate, in TFLOP/s (algorithmic FLOPs: the causal half only).  The same
-JSON line carries the split-KV decode workloads (ragged bf16 64K-128K cache; FP8 E4M3, INT8 and
-INT4 caches of 32768 tokens; paged and multi-token variants) in KV GB/s and the packed varlen
-prefill, each against the measured roofline, the oracle timed on the host cores, and an
-end-to-end number through host buffers.
+bf16 in / fp32 accumulate, in TFLOP/s (algorithmic FLOPs: the causal half only), printed last.
+Before it, one compact JSON line per secondary workload: the split-KV decodes (ragged bf16
+64K-128K cache; FP8 E4M3, INT8 and INT4 caches of 32768 tokens; paged and multi-token variants)
+in KV GB/s, the packed varlen prefill, and the streamed causal prefill over 2^20 host-resident
+tokens, each against the measured roofline and the oracle timed on the host cores; the headline
+line repeats them as a summary.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--stream]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-stream]
 
 Under torchrun (N > 1) every rank runs the same workload on its own GPU (independent
 replicas: weak scaling, no collective on the data path); the time is the max over ranks.
@@ -422,26 +423,65 @@ def varlen_oracle_sample(w, d):
 
 
 def bench_stream(dev, pk):
+    """The streamed causal prefill over 2^20 host-resident tokens (attn_chunked_stream: pinned host
+    Q/K/V/O/LSE, 64K-token key chunks, 16e9-byte device budget), run once.  Reports TFLOP/s over the
+    device span from the first upload to the end of the last copy back, the prefill tasks' own rate
+    against the tensor roofline, copy-engine GB/s of each direction (bytes / summed copy time), and
+    the overlap fraction (compute time / device span: 1 = every copy hidden)."""
     from exact_long_context_tmem_b200 import attn as A
 
     w = I.WORKLOADS[STREAM]
     g = I.generator(w.seed)
     shape_q = (w.B, w.S, w.Hq, w.D)
     shape_kv = (w.B, w.S, w.Hkv, w.D)
+    t_gen = time.perf_counter()
     q = I.randn_bf16(shape_q, g, out=torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True))
     k = I.randn_bf16(shape_kv, g, out=torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True))
     v = I.randn_bf16(shape_kv, g, out=torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True))
     o = torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)
     lse = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, pin_memory=True)
+    t_gen = time.perf_counter() - t_gen
     _, _, st = A.attn_chunked_stream(q, k, v, causal=True, chunk_tokens=w.chunk_tokens, budget_bytes=w.budget_bytes,
                                      o_h=o, lse_h=lse)
     flops = prefill_flops(w)
-    return {"workload": STREAM, "value": round(flops / (st.ms_total * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
-            "ms_total": round(st.ms_total, 1), "q_block": st.plan.q_block, "kv_chunk": st.plan.kv_chunk,
-            "tasks": st.plan.n_tasks, "device_bytes": st.plan.device_bytes,
-            "h2d_GBps": round(st.h2d_bytes / (st.ms_total * 1e-3) / 1e9, 2),
-            "d2h_GBps": round(st.d2h_bytes / (st.ms_total * 1e-3) / 1e9, 2),
-            "h2d_bytes": st.h2d_bytes, "d2h_bytes": st.d2h_bytes}
+    tf = flops / (st.ms_device * 1e-3) / 1e12
+    busy_tf = flops / (st.ms_compute_busy * 1e-3) / 1e12
+    line = {"workload": STREAM, "value": round(tf, 1), "unit": "TFLOP/s", "ms_per_step": round(st.ms_device, 1),
+            "flops_per_step": flops, "q_block": st.plan.q_block, "kv_chunk": st.plan.kv_chunk,
+            "tasks": st.plan.n_tasks, "device_bytes": st.plan.device_bytes, "device_budget": w.budget_bytes,
+            "roofline": {"bound": "tensor", "achieved": round(busy_tf, 1), "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(busy_tf / pk["bf16_tflops"], 4), "traffic": None,
+                         "timed": "prefill tasks + block finishes, summed CUDA-event time on the compute stream"},
+            "copies": {"h2d_GBps": round(st.h2d_bytes / (st.ms_h2d * 1e-3) / 1e9, 2),
+                       "d2h_GBps": round(st.d2h_bytes / (st.ms_d2h * 1e-3) / 1e9, 2),
+                       "h2d_bytes": st.h2d_bytes, "d2h_bytes": st.d2h_bytes,
+                       "ms_h2d": round(st.ms_h2d, 1), "ms_d2h": round(st.ms_d2h, 1),
+                       "timed": "summed CUDA-event time of each copy batch on its stream"},
+            "overlap": round(st.ms_compute_busy / st.ms_device, 4),
+            "ms_compute_busy": round(st.ms_compute_busy, 1), "ms_call_wall": round(st.ms_total, 1),
+            "e2e": {"value": round(tf, 1), "unit": "TFLOP/s", "h2d_bytes_per_step": st.h2d_bytes,
+                    "d2h_bytes_per_step": st.d2h_bytes},
+            "launches": 2 * st.plan.n_tasks, "input_gen_s": round(t_gen, 1),
+            "cpu_baseline": stream_oracle_sample(w, q, k, v)}
+    return line
+
+
+def stream_oracle_sample(w, q, k, v, n_rows=4):
+    """Time the float64 oracle on a bounded sample of the streamed workload: n_rows query rows
+    from the end of the sequence (each sees about 2^20 keys) for the 4 query heads of KV head 0
+    (the widening of that head's K and V to float64 inside the timed region).  TFLOP/s counts the
+    causal pairs as the GPU line does."""
+    from oracle import attention as O
+
+    G = w.Hq // w.Hkv
+    step = max(1, w.chunk_tokens or w.S // (n_rows + 1))
+    rows = [r for r in (w.S - 1 - i * step for i in range(n_rows)) if r >= 0]
+    t = time.perf_counter()
+    O.attention(q[:, :, :G], k[:, :, :1], v[:, :, :1], scale=w.scale, causal=True, rows=rows)
+    dt = time.perf_counter() - t
+    flops = sum(4.0 * w.D * (r + 1) for r in rows) * G
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
+            "sample": f"{n_rows} query rows near the end x {G} heads of KV head 0 ({dt:.1f} s)"}
 
 
 # ------------------------------------------------------------------ oracle (CPU baseline)
@@ -519,12 +559,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--stream", action="store_true", help="also run the 1M-token streamed prefill")
+    ap.add_argument("--no-stream", action="store_true", help="leave out the 1M-token streamed prefill")
     ap.add_argument("--cpu-rows", type=int, default=128)
     ap.add_argument("--workloads",
                     default="prefill,prefill_varlen,decode_bf16,decode_fp8,decode_bf16_paged,decode_fp8_paged,"
-                            "decode_bf16_multi,decode_fp8_multi,decode_int8,decode_int4",
-                    help="comma list of prefill, prefill_varlen, decode_{bf16,fp8,int8,int4}[_paged|_multi] "
+                            "decode_bf16_multi,decode_fp8_multi,decode_int8,decode_int4,stream",
+                    help="comma list of prefill, prefill_varlen, stream, decode_{bf16,fp8,int8,int4}[_paged|_multi] "
                          "(profiling runs select one)")
     args = ap.parse_args()
     w = I.WORKLOADS[HEADLINE]
@@ -566,25 +606,43 @@ def main():
     A.lib()
     pk = peaks()
     sel = set(args.workloads.split(","))
+
+    def emit(line):
+        """A secondary workload: its own compact JSON line, printed before the headline line."""
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "kind": "secondary", "n_gpus": world, **line}), flush=True)
+
     pre = bench_prefill(w, args.steps, args.warmup, world, dev, pk) if "prefill" in sel else None
-    dec = []
+    summary = {}
+
+    def note(line):
+        summary[line["workload"]] = [line["value"], line["unit"], line["roofline"]["frac"]]
+        emit(line)
+
     if not args.no_decode:
         for key, name in DECODE_WORKLOADS:
             if key in sel:
-                dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk))
+                note(bench_decode(name, args.steps, args.warmup, world, dev, pk))
             if key + "_paged" in sel:
-                dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk, paged=True))
+                note(bench_decode(name, args.steps, args.warmup, world, dev, pk, paged=True))
             if key + "_multi" in sel:
-                dec.append(bench_decode(name, args.steps, args.warmup, world, dev, pk, n_q=4))
-    varlen = bench_prefill_varlen(args.steps, args.warmup, world, dev, pk) if "prefill_varlen" in sel else None
+                note(bench_decode(name, args.steps, args.warmup, world, dev, pk, n_q=4))
+    if "prefill_varlen" in sel:
+        note(bench_prefill_varlen(args.steps, args.warmup, world, dev, pk))
     st, site = A.attn_device_status(reset=True)
     if st != 0:
         raise SystemExit(f"device status {st} at wait site {site}")
-    stream = bench_stream(dev, pk) if args.stream and rank == 0 else None
+    # The streamed 2^20-token prefill holds ~20 GiB of pinned host memory and takes ~10 s: one run,
+    # on a single process (with several replicas it is left out).
+    if "stream" in sel and not args.no_stream:
+        if world == 1:
+            note(bench_stream(dev, pk))
+        elif rank == 0:
+            summary[STREAM] = "left out with more than one process (host memory)"
     cpu = None
     if pre is None:
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "partial": True, "decode": dec, "prefill_varlen": varlen}), flush=True)
+            print(json.dumps({"metric": METRIC, "partial": True, "summary": summary}), flush=True)
         return
     if rank == 0 and world == 1:
         tf, dt, rows = oracle_sample(w, args.cpu_rows)
@@ -597,7 +655,7 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic N(0,1), seeded", "config": config, "roofline": pre["roofline"],
                 "cpu_baseline": cpu, "e2e": pre["e2e"], "clocks": pre["clocks"], "gpu_launches": pre["launches"],
-                "decode": dec, "prefill_varlen": varlen, "stream": stream}
+                "summary": summary}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -68,7 +68,8 @@ class StreamPlan(ctypes.Structure):
 
 class StreamStats(ctypes.Structure):
     _fields_ = [("plan", StreamPlan), ("h2d_bytes", ctypes.c_longlong), ("d2h_bytes", ctypes.c_longlong),
-                ("ms_total", ctypes.c_double), ("ms_compute", ctypes.c_double)]
+                ("ms_total", ctypes.c_double), ("ms_compute", ctypes.c_double), ("ms_device", ctypes.c_double),
+                ("ms_compute_busy", ctypes.c_double), ("ms_h2d", ctypes.c_double), ("ms_d2h", ctypes.c_double)]
 
 
 _lib = None

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "internal.h"
 #include "decode.cuh"
 #include "decode_fp8.cuh"
 #include "decode_int.cuh"
@@ -126,7 +127,8 @@ template <int D>
 static attn_status_t launch_prefill(const void* q, const void* k, const void* v, void* o, int o_f32, float* lse,
                                     const attn_dims_t& d, int S, int T, int causal, long long q_pos0,
                                     long long kv_pos0, cudaStream_t stream, const int* cu_q = nullptr,
-                                    const int* cu_k = nullptr, int max_s = 0, const long long* strides = nullptr) {
+                                    const int* cu_k = nullptr, int max_s = 0, const long long* strides = nullptr,
+                                    int accumulate = 0) {
   using C = PrefillCfg<D>;
   static std::atomic<uint64_t> smem_done{0};
   static std::atomic<int> regs_state{0};
@@ -181,6 +183,7 @@ static attn_status_t launch_prefill(const void* q, const void* k, const void* v,
   p.o_ss = strides ? strides[10] : (long long)d.Hq * D;
   p.o_sh = strides ? strides[11] : (long long)D;
   p.lse = lse;
+  p.accumulate = accumulate;
   p.cu_q = cu_q;
   p.cu_k = cu_k;
   if (p.n_items == 0) return ATTN_OK;
@@ -532,6 +535,30 @@ attn_status_t attn_prefill_varlen(const void* q, const void* k, const void* v, v
   return launch_prefill<64>(q, k, v, o, f32, lse, dims, total_q, total_k, causal, 0, 0, st, cu_seqlens_q,
                             cu_seqlens_k, max_seqlen_q);
 }
+
+}  // extern "C"
+
+namespace attn {
+
+attn_status_t prefill_accumulate_f32(const void* q, const void* k, const void* v, float* o, float* lse,
+                                     attn_dims_t dims, int S, int T, int causal, long long q_pos0, long long kv_pos0,
+                                     void* stream) {
+  if (!dims_ok(dims) || S < 0 || T < 0 || q_pos0 < 0 || kv_pos0 < 0) return ATTN_ERR_INVALID_ARG;
+  if (dims.B == 0 || S == 0 || T == 0) return ATTN_OK;  // no key: every stored partial stands
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return ATTN_ERR_INVALID_ARG;
+  if (dims.D != 64 && dims.D != 128) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims.D == 128)
+    return launch_prefill<128>(q, k, v, o, 1, lse, dims, S, T, causal, q_pos0, kv_pos0, st, nullptr, nullptr, 0,
+                               nullptr, 1);
+  return launch_prefill<64>(q, k, v, o, 1, lse, dims, S, T, causal, q_pos0, kv_pos0, st, nullptr, nullptr, 0, nullptr,
+                            1);
+}
+
+}  // namespace attn
+
+extern "C" {
 
 int attn_decode_num_splits(attn_dims_t dims, int Tmax, int num_splits) {
   if (!dims_ok(dims) || Tmax < 0) return 0;

@@ -42,6 +42,10 @@ struct PrefillParams {
   int o_f32;
   long long o_sb, o_ss, o_sh;  // element strides of o between batches, tokens and heads (D contiguous)
   float* lse;
+  // 1: o (float32) and lse already hold the normalised output and log-sum-exp of earlier key chunks
+  // for these rows; the kernel merges its own result into them by log-sum-exp (the exact merge of
+  // partial softmax states), and leaves rows that see no key here unchanged.
+  int accumulate;
   // Packed variable-length batch (ORT packed-QSA analysis, "Code analysis": cumulative sequence
   // lengths, and a token's position = past length + its index among the new tokens): sequence b's
   // queries are rows cu_q[b] .. cu_q[b+1]-1 of q/o/lse and its keys rows cu_k[b] .. cu_k[b+1]-1 of
@@ -223,13 +227,13 @@ __global__ void __launch_bounds__(384, 1)
         const int st = j % C::NST;
         const uint32_t ph = (j / C::NST) & 1;
         ATTN_TRACE_AT(0, 4, j);
-        if (!mbar_wait(&k_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; break; }
+        if (!mbar_wait<true>(&k_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; break; }
         mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d_hint(smem + C::OFF_K + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmK, &k_full[st], bx * 64,
                            it.kvh, it.k_base + j * 128, it.bc, pol_kv);
         ATTN_TRACE_AT(0, 5, j);
-        if (!mbar_wait(&v_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; issued = 2 * j + 1; break; }
+        if (!mbar_wait<true>(&v_empty[st], ph ^ 1, SITE_PF_LOAD_EMPTY)) { ok = false; issued = 2 * j + 1; break; }
         mbar_arrive_expect_tx(&v_full[st], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d_hint(smem + C::OFF_V + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmV, &v_full[st], bx * 64,
@@ -239,12 +243,12 @@ __global__ void __launch_bounds__(384, 1)
       ATTN_TRACE_AT(0, 6, issued);
       if (!ok) {
         // Let every copy already issued land before the CTA's shared memory is released.
-        mbar_wait_drain(q_full, 0, SITE_PF_DRAIN);
+        mbar_wait_drain<true>(q_full, 0, SITE_PF_DRAIN);
         const int nk = (issued + 1) / 2, nv = issued / 2;
         for (int j = (nk > C::NST ? nk - C::NST : 0); j < nk; ++j)
-          mbar_wait_drain(&k_full[j % C::NST], (j / C::NST) & 1, SITE_PF_DRAIN);
+          mbar_wait_drain<true>(&k_full[j % C::NST], (j / C::NST) & 1, SITE_PF_DRAIN);
         for (int j = (nv > C::NST ? nv - C::NST : 0); j < nv; ++j)
-          mbar_wait_drain(&v_full[j % C::NST], (j / C::NST) & 1, SITE_PF_DRAIN);
+          mbar_wait_drain<true>(&v_full[j % C::NST], (j / C::NST) & 1, SITE_PF_DRAIN);
       }
     }
     __syncwarp();
@@ -281,10 +285,10 @@ __global__ void __launch_bounds__(384, 1)
                        (acc || kk > 0) ? 1u : 0u);
       };
       if (lane == 0) ATTN_TRACE_AT(1, 3, 0);
-      bool ok = mbar_wait_warp(q_full, 0, SITE_PF_MMA_Q);
+      bool ok = mbar_wait_warp<true>(q_full, 0, SITE_PF_MMA_Q);
       if (lane == 0) ATTN_TRACE_AT(1, 4, ok);
       if (ok && n > 0) {
-        ok = mbar_wait_warp(&k_full[0], 0, SITE_PF_MMA_K);
+        ok = mbar_wait_warp<true>(&k_full[0], 0, SITE_PF_MMA_K);
         if (ok) {
           tc_fence_after();
           if (lane == 0) ATTN_EVT(0, 0);
@@ -303,22 +307,22 @@ __global__ void __launch_bounds__(384, 1)
         const int st1 = (j + 1) % C::NST;
         const uint32_t ph1 = ((j + 1) / C::NST) & 1;
         if (lane == 0) ATTN_TRACE_AT(1, 5, j);
-        if (!(ok = mbar_wait_warp(&v_full[st], ph, SITE_PF_MMA_V))) break;
+        if (!(ok = mbar_wait_warp<true>(&v_full[st], ph, SITE_PF_MMA_V))) break;
         if (lane == 0) ATTN_TRACE_AT(1, 6, j);
-        if (!(ok = mbar_wait_warp(&p_full[0], j & 1, SITE_PF_MMA_P))) break;
+        if (!(ok = mbar_wait_warp<true>(&p_full[0], j & 1, SITE_PF_MMA_P))) break;
         if (lane == 0) ATTN_TRACE_AT(1, 7, j);
         tc_fence_after();
         if (lane == 0) ATTN_EVT(j, 3);
         issue_pv(0, st, j > 0);
         if (more) {
-          if (!(ok = mbar_wait_warp(&k_full[st1], ph1, SITE_PF_MMA_K))) break;
+          if (!(ok = mbar_wait_warp<true>(&k_full[st1], ph1, SITE_PF_MMA_K))) break;
           tc_fence_after();
           if (lane == 0) ATTN_EVT(j + 1, 0);
           issue_qk(0, st1);
           mma_commit_elect(&s_full[0]);
         }
         if (lane == 0) ATTN_TRACE_AT(1, 8, j);
-        if (!(ok = mbar_wait_warp(&p_full[1], j & 1, SITE_PF_MMA_P))) break;
+        if (!(ok = mbar_wait_warp<true>(&p_full[1], j & 1, SITE_PF_MMA_P))) break;
         if (lane == 0) ATTN_TRACE_AT(1, 9, j);
         tc_fence_after();
         if (lane == 0) ATTN_EVT(j, 11);
@@ -335,7 +339,7 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) ATTN_TRACE_AT(1, 10, ok);
       // Drain: every MMA issued above completes before TMEM is released.
       mma_commit_elect(drain);
-      const bool drained = mbar_wait_drain(drain, 0, SITE_PF_DRAIN);
+      const bool drained = mbar_wait_drain<true>(drain, 0, SITE_PF_DRAIN);
       if (lane == 0) ATTN_TRACE_AT(1, 11, drained);
     }
     __syncwarp();
@@ -357,7 +361,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < n; ++j) {
       if (r == 0) ATTN_TRACE_AT(2 + slot, 1, j);
       // tcgen05.ld/st are warp-collective: every lane takes the same branch around them.
-      if (!(ok = mbar_wait_warp(&s_full[slot], j & 1, SITE_PF_SM_S))) break;
+      if (!(ok = mbar_wait_warp<true>(&s_full[slot], j & 1, SITE_PF_SM_S))) break;
       if (r == 0) ATTN_TRACE_AT(2 + slot, 2, j);
       if (r == 0) ATTN_EVT(j, slot * 8 + 1);
       tc_fence_after();
@@ -466,12 +470,29 @@ __global__ void __launch_bounds__(384, 1)
     const bool have_o = n > 0;
     if (r == 0) ATTN_TRACE_AT(4 + slot, 1, ok);
     if (ok && have_o) {
-      ok = mbar_wait_warp(o_full, 0, SITE_PF_EPI_O);
+      ok = mbar_wait_warp<true>(o_full, 0, SITE_PF_EPI_O);
       tc_fence_after();
     }
     if (r == 0) ATTN_TRACE_AT(4 + slot, 2, ok);
     if (ok) {
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      float lse = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const long long lse_idx = (it.lse_row0 + row) * p.Hq + it.head[slot];
+      float w_old = 0.f;   // weight of the stored partial (accumulate)
+      bool store = row_ok;
+      if (p.accumulate && row_ok) {
+        const float lse_old = p.lse[lse_idx];
+        if (lse == -INFINITY) {
+          store = false;  // no key of this chunk is visible: the stored partial stands
+        } else if (lse_old != -INFINITY) {
+          const float mx = fmaxf(lse_old, lse);
+          const float e_old = expf(lse_old - mx), e_new = expf(lse - mx);
+          const float inv = 1.f / (e_old + e_new);
+          w_old = e_old * inv;
+          inv_l *= e_new * inv;
+          lse = mx + logf(e_old + e_new);
+        }
+      }
       const long long orow = it.o_base + (long long)row * p.o_ss + (long long)it.head[slot] * p.o_sh;
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -482,14 +503,26 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;
         }
-        if (!row_ok) continue;
+        if (!store) continue;
         if (p.o_f32) {
           float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + orow + c * 32);
+          if (w_old != 0.f) {  // the stored partial is read only when it has a weight
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            st_global_cs_v4f(dst + i, make_float4(__uint_as_float(v[4 * i]) * inv_l, __uint_as_float(v[4 * i + 1]) * inv_l,
-                                                  __uint_as_float(v[4 * i + 2]) * inv_l,
-                                                  __uint_as_float(v[4 * i + 3]) * inv_l));
+            for (int i = 0; i < 8; ++i) {
+              const float4 old = dst[i];
+              dst[i] = make_float4(fmaf(__uint_as_float(v[4 * i]), inv_l, w_old * old.x),
+                                   fmaf(__uint_as_float(v[4 * i + 1]), inv_l, w_old * old.y),
+                                   fmaf(__uint_as_float(v[4 * i + 2]), inv_l, w_old * old.z),
+                                   fmaf(__uint_as_float(v[4 * i + 3]), inv_l, w_old * old.w));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              st_global_cs_v4f(dst + i, make_float4(__uint_as_float(v[4 * i]) * inv_l,
+                                                    __uint_as_float(v[4 * i + 1]) * inv_l,
+                                                    __uint_as_float(v[4 * i + 2]) * inv_l,
+                                                    __uint_as_float(v[4 * i + 3]) * inv_l));
+          }
         } else {
           uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) + orow + c * 32);
 #pragma unroll
@@ -503,10 +536,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (p.lse && row_ok) {
-        const float lse = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        p.lse[(it.lse_row0 + row) * p.Hq + it.head[slot]] = lse;
-      }
+      if (p.lse && store) p.lse[lse_idx] = lse;
     }
   }
   tc_fence_before();

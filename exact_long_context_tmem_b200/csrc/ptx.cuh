@@ -71,9 +71,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // past the deadline the wait records ATTN_ERR_TIMEOUT with a site code in the
 // device status word and returns false, and the caller unwinds.
 // A drain wait (for copies or MMAs this thread already issued, which complete on their own)
-// ignores errors recorded by other roles and only stops at the time limit.  Inlined: a call
-// across warpgroups that trade registers (setmaxnreg) cannot be register-allocated.
-__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int site, bool drain) {
+// ignores errors recorded by other roles and only stops at the time limit.
+__device__ __forceinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, int site, bool drain) {
   const uint64_t t0 = globaltimer_ns();
   const uint64_t limit = g_wait_limit_ns;
   for (uint32_t it = 0;; ++it) {
@@ -88,21 +87,30 @@ __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, i
   }
 }
 
+// The slow path out of line (kernels whose hot loops stay small), or inlined (kernels whose
+// warpgroups trade registers with setmaxnreg: a call across such regions cannot be register-allocated).
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int site, bool drain) {
+  return mbar_wait_loop(bar, parity, site, drain);
+}
+
+template <bool INL = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, site, false);
+  return INL ? mbar_wait_loop(bar, parity, site, false) : mbar_wait_slow(bar, parity, site, false);
 }
 
 // Wait for roles in which all 32 lanes run the same code: the outcome is made warp-uniform, so a
 // timeout never splits a warp in front of a warp-collective tcgen05 instruction.
+template <bool INL = false>
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int site) {
-  const bool ok = mbar_wait(bar, parity, site);
+  const bool ok = mbar_wait<INL>(bar, parity, site);
   return __all_sync(0xffffffffu, ok);
 }
 
+template <bool INL = false>
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int site) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, site, true);
+  return INL ? mbar_wait_loop(bar, parity, site, true) : mbar_wait_slow(bar, parity, site, true);
 }
 
 // ---------------------------------------------------------------- fences

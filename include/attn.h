@@ -276,9 +276,10 @@ ATTN_API attn_status_t attn_merge_lse(const float* o_parts, const float* lse_par
  * [CQSA] Methodology 2-4: attention is split into independent sub-tasks — here (query block,
  * key chunk) rectangles that cover every visible (query, key) pair exactly once — queued and
  * streamed host->device on a copy stream, computed on the compute stream, and recombined by
- * the log-sum-exp merge; finished blocks are swapped back to host memory.  A controller picks
- * the block sizes from the budget ([CQSA] Methodology 4; its Limitations section calls the
- * block-size rule a plain heuristic).
+ * the log-sum-exp merge (inside each task's kernel); finished blocks are swapped back to host
+ * memory on a stream of their own.  A controller picks the block sizes from the budget ([CQSA]
+ * Methodology 4; its Limitations section calls the block-size rule a plain heuristic): the query
+ * block that fits and sends the fewest key chunks across the host link.
  *
  *   q_h, k_h, v_h  host bf16 [B, S, Hq, D] / [B, S, Hkv, D]; pinned memory lets copies overlap
  *   o_h            host bf16 [B, S, Hq, D];  lse_h host float32 [B, S, Hq] or NULL
@@ -296,12 +297,18 @@ typedef struct {
   long long device_bytes; /* bytes the plan allocates on the device */
 } attn_stream_plan_t;
 
+/* Timings are CUDA-event times on the stream that runs each step (0 when the call failed). */
 typedef struct {
   attn_stream_plan_t plan;
   long long h2d_bytes;     /* host->device bytes copied */
   long long d2h_bytes;     /* device->host bytes copied */
-  double ms_total;         /* wall time of the call (host clock) */
-  double ms_compute;       /* summed device time of prefill + merge launches (CUDA events) */
+  double ms_total;         /* wall time of the call (host clock), set-up and frees included */
+  double ms_compute;       /* compute stream, from its first launch to its last */
+  double ms_device;        /* device span from the first upload to the end of the last copy back */
+  double ms_compute_busy;  /* summed time of the compute steps (prefill tasks and block finishes):
+                              the span the call would take with every copy hidden */
+  double ms_h2d;           /* summed time of the host->device copies (copy stream) */
+  double ms_d2h;           /* summed time of the device->host copies (their own stream) */
 } attn_stream_stats_t;
 
 ATTN_API attn_status_t attn_stream_plan(attn_dims_t dims, long long S, int causal, long long chunk_tokens,

@@ -97,3 +97,16 @@ def test_scale_shape_is_checked():
         A._check_kv_rows(k, k, D, A.ATTN_INT8, ok.double(), ok)
     with pytest.raises(ValueError):
         A._check_kv_rows(k, k, D, A.ATTN_INT8, ok, torch.empty((2, 3, 4), dtype=torch.float32))
+
+
+def test_bench_stream_oracle_sample():
+    """The streamed workload's CPU baseline runs the oracle on rows near the end of the sequence for
+    the query heads of KV head 0, from the same host tensors."""
+    w = I.Workload("s", "stream", B=1, Hq=8, Hkv=2, D=64, S=700, T=700, chunk_tokens=128, seed=3)
+    g = I.generator(w.seed)
+    q = I.randn_bf16((1, w.S, w.Hq, w.D), g)
+    k = I.randn_bf16((1, w.S, w.Hkv, w.D), g)
+    v = I.randn_bf16((1, w.S, w.Hkv, w.D), g)
+    cb = bench.stream_oracle_sample(w, q, k, v, n_rows=3)
+    assert cb["kind"] == "oracle" and cb["unit"] == "TFLOP/s" and cb["value"] > 0
+    assert "3 query rows" in cb["sample"] and "4 heads" in cb["sample"]
