@@ -187,7 +187,11 @@ static attn_status_t launch_prefill(const void* q, const void* k, const void* v,
   p.cu_q = cu_q;
   p.cu_k = cu_k;
   if (p.n_items == 0) return ATTN_OK;
-  prefill_fwd_sm100<D><<<p.n_items, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  // Persistent: one CTA per SM (shared memory and TMEM allow one), at most one per work item.
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min(p.n_items, std::max(sms, 1));
+  prefill_fwd_sm100<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   ATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
 }
