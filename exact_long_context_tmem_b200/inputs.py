@@ -69,6 +69,9 @@ WORKLOADS = {
     "stream_b1_h32g8_d128_s1m_chunk64k": Workload(
         "stream_b1_h32g8_d128_s1m_chunk64k", "stream", B=1, Hq=32, Hkv=8, D=128,
         S=1 << 20, T=1 << 20, chunk_tokens=65536, budget_bytes=16 * 10**9, seed=1004),
+    "stream_b1_h32g8_d128_s128k_chunk16k": Workload(
+        "stream_b1_h32g8_d128_s128k_chunk16k", "stream", B=1, Hq=32, Hkv=8, D=128, S=131072, T=131072,
+        chunk_tokens=16384, budget_bytes=2_500_000_000, seed=1005),
 }
 
 

@@ -163,3 +163,17 @@ def test_prefill_strided_no_visible_keys(cuda_device):
     assert_o_close(o, ro)
     assert_lse_close(to_np(lse).transpose(0, 2, 1), rl)
     device_clean()
+
+
+def test_prefill_more_items_than_the_schedule_holds(cuda_device):
+    """80000 one-token sequences make 80000 work items, more than the 512 per CTA the kernel's
+    schedule list holds at 148 CTAs: every CTA falls back to taking every grid-th item, and every
+    row is still computed (one visible key: O = V, LSE = scale * q.k)."""
+    B, D = 80000, 64
+    q, k, v = _gen(B, 1, 1, 1, 1, D, seed=25)
+    o, lse = A.attn_prefill(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), causal=True)
+    torch.cuda.synchronize()
+    ro, rl = O.attention(q, k, v, scale=1 / math.sqrt(D), causal=True)
+    assert_o_close(o, ro)
+    assert_lse_close(to_np(lse).transpose(0, 2, 1), rl)
+    device_clean()
