@@ -229,8 +229,10 @@ template <int GP, bool MULTI>
 __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const DecodeParams& p, int G, int split,
                                                 int kvh, int b, int lane, int wq, int t, uint32_t tO_lane,
                                                 float* red_sum, uint64_t* sum_bar, uint32_t sum_parity,
-                                                uint64_t* o_final, uint32_t o_parity, uint64_t* o_free) {
+                                                uint64_t* o_final, uint32_t o_parity, uint64_t* o_free,
+                                                int d_out = -1) {
   constexpr int D = 128;
+  if (d_out < 0) d_out = t;  // the head-dimension element that TMEM lane t of O^T holds
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
     const float s = warp_sum(rows.l_part[g]);
@@ -259,9 +261,9 @@ __device__ __forceinline__ bool decode_epilogue(DecodeRows<GP>& rows, const Deco
       if (g == t) my_lse = lse;
       const long long h = MULTI ? decode_row_index(p, b, kvh, g) : (long long)b * p.Hq + (long long)kvh * p.G + g;
       if (p.n_splits == 1) {
-        p.o[h * D + t] = __float2bfloat16_rn(ov);
+        p.o[h * D + d_out] = __float2bfloat16_rn(ov);
       } else {
-        p.o_part[((long long)split * rows_all + h) * D + t] = ov;
+        p.o_part[((long long)split * rows_all + h) * D + d_out] = ov;
       }
     }
   }

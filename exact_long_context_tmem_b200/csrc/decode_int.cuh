@@ -90,22 +90,36 @@ __device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t& h01, uint32_t&
   h23 = sub_f16x2(__byte_perm(u, 0x64646464u, 0x5352u), 0x64806480u);
 }
 
-// Eight INT4 codes (one word; element k in nibble k) -> four f16 pairs in element order, exact:
-// code + 8 becomes the low 4 mantissa bits of an f16 in [1024, 1040); 1032 is subtracted.
-__device__ __forceinline__ void i4x8_to_f16(uint32_t w, uint32_t* h) {
-  const uint32_t u = w ^ 0x88888888u;
-  const uint32_t a = (u & 0x000F000Fu) | 0x64006400u;          // elements 0, 4
-  const uint32_t b = ((u >> 4) & 0x000F000Fu) | 0x64006400u;   // 1, 5
-  const uint32_t c = ((u >> 8) & 0x000F000Fu) | 0x64006400u;   // 2, 6
-  const uint32_t d = ((u >> 12) & 0x000F000Fu) | 0x64006400u;  // 3, 7
-  h[0] = sub_f16x2(__byte_perm(a, b, 0x5410u), 0x64086408u);
-  h[1] = sub_f16x2(__byte_perm(c, d, 0x5410u), 0x64086408u);
-  h[2] = sub_f16x2(__byte_perm(a, b, 0x7632u), 0x64086408u);
-  h[3] = sub_f16x2(__byte_perm(c, d, 0x7632u), 0x64086408u);
+__device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) ^ c
+  return d;
+}
+__device__ __forceinline__ uint32_t fma_f16x2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
+// Eight INT4 codes (one word; element k in nibble k) -> four f16 pairs (0,4), (1,5), (2,6), (3,7),
+// exact, in five integer instructions: one lop3 per pair puts code + 8 (the nibble with its top bit
+// flipped) into the mantissa of an f16 in [1024, 1040) (low nibbles) or, at 16x, in [1024, 1264)
+// (high nibbles), which a subtraction or an fma by 1/16 takes back to the code.  The pairing is not
+// element order: a kernel using it permutes the other operand of each product the same way.
+__device__ __forceinline__ void i4x8_to_f16_paired(uint32_t w, uint32_t* h) {
+  const uint32_t w8 = w >> 8;
+  h[0] = sub_f16x2(lop3_and_xor(w, 0x000F000Fu, 0x64086408u), 0x64086408u);                // 0, 4
+  h[1] = fma_f16x2(lop3_and_xor(w, 0x00F000F0u, 0x64806480u), 0x2C002C00u, 0xD480D480u);   // 1, 5
+  h[2] = sub_f16x2(lop3_and_xor(w8, 0x000F000Fu, 0x64086408u), 0x64086408u);               // 2, 6
+  h[3] = fma_f16x2(lop3_and_xor(w8, 0x00F000F0u, 0x64806480u), 0x2C002C00u, 0xD480D480u);  // 3, 7
+}
+
+// Position within each group of eight head-dimension elements of the INT4 path: the f16 pair at
+// positions (2i, 2i+1) holds elements (i, i + 4).  Element of position q: (q >> 1) + 4 (q & 1).
+__device__ __forceinline__ int int4_paired_element(int q) { return (q & ~7) | (((q & 7) >> 1) + 4 * (q & 1)); }
+
 // Elements [64 half, 64 half + 64) of token row t of a code tile as 32 f16 pairs (zeros when the
-// token is not valid).
+// token is not valid); INT4 rows come out in the paired order of i4x8_to_f16_paired.
 template <int BITS>
 __device__ __forceinline__ void int_row_half_to_f16(const uint8_t* tile, int t, int half, bool valid,
                                                     uint32_t (&h)[32]) {
@@ -118,7 +132,7 @@ __device__ __forceinline__ void int_row_half_to_f16(const uint8_t* tile, int t, 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       if (BITS == 8) i8x4_to_f16(wd[i], h[k * 8 + 2 * i], h[k * 8 + 2 * i + 1]);
-      else i4x8_to_f16(wd[i], &h[k * 16 + 4 * i]);
+      else i4x8_to_f16_paired(wd[i], &h[k * 16 + 4 * i]);
     }
   }
 }
@@ -148,6 +162,7 @@ __device__ __forceinline__ long long int_scale_index(const DecodeParams& p, int 
 // [-100, 100]) into the 128B-swizzled K-major B operand (two 64-wide boxes of 16 rows); 2^-e of
 // row g goes to qsc[g].  128 threads: chunk c = tid + 128 k is row c / 16, elements 8 (c % 16)..,
 // so the 16 threads of a row are 16 consecutive lanes of one warp.
+template <int BITS>
 __device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kvh, int b, int tid, uint8_t* q_smem,
                                             float* qsc) {
 #pragma unroll
@@ -171,7 +186,10 @@ __device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kv
     const float up = __uint_as_float((uint32_t)(e + 127) << 23);
     uint32_t hv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) hv[i] = pack_f16x2(f[2 * i] * up, f[2 * i + 1] * up);
+    for (int i = 0; i < 4; ++i) {
+      if (BITS == 8) hv[i] = pack_f16x2(f[2 * i] * up, f[2 * i + 1] * up);
+      else hv[i] = pack_f16x2(f[i] * up, f[i + 4] * up);  // the paired order of the INT4 K rows
+    }
     *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * (16 * 128) + sw128_offset(g, cc & 7)) =
         make_uint4(hv[0], hv[1], hv[2], hv[3]);
     if (cc == 0) qsc[g] = __uint_as_float((uint32_t)(127 - e) << 23);
@@ -490,7 +508,7 @@ __global__ void __launch_bounds__(512, 1)
     const int wg_tid = threadIdx.x - 320;
     for (int i = wg_tid; i < NB * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
-    int_stage_q(p, G, kvh, b, wg_tid, smem + C::OFF_Q, qsc);
+    int_stage_q<BITS>(p, G, kvh, b, wg_tid, smem + C::OFF_Q, qsc);
     fence_proxy_async_smem();
     warp_arrive(q_ready, lane);
     named_barrier_sync(1, 128);  // every row's 2^-e is in qsc
@@ -571,7 +589,7 @@ __global__ void __launch_bounds__(512, 1)
     if (t == 0) ATTN_EVT(63, 2);
     if (ok)
       decode_epilogue<GP, false>(rows, p, G, split, kvh, b, lane, wq, t, tO + lane_off, red_sum, sum_bar, 0, o_final,
-                                 0, nullptr);
+                                 0, nullptr, BITS == 4 ? int4_paired_element(t) : t);  // O^T lane t: V's paired order
     if (t == 0) ATTN_EVT(63, 3);
   }
   tc_fence_before();

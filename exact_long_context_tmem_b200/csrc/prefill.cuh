@@ -5,10 +5,9 @@
 // compute the score block, update the running row max and row sum (online softmax), and
 // accumulate P.V into the output; the S x T score matrix never leaves the SM.
 //
-// Persistent: one CTA per SM works through the items dealt to it (heaviest causal tiles first,
-// balanced across CTAs); TMEM stays allocated and every barrier keeps counting phases across
-// items, so the next item's first QK^T overlaps the current epilogue and the K/V ring never
-// drains between items.
+// Persistent: one CTA per SM walks the work items c, c + grid, ... (heaviest causal tiles first);
+// TMEM stays allocated and every barrier keeps counting phases across items, so the next item's
+// first QK^T overlaps the current epilogue and the K/V ring never drains between items.
 //
 // Roles (384 threads; warpgroup 0 hands most of its registers to warpgroups 1 and 2):
 //   warp 0        TMA producer: per item the Q tiles, then K_j / V_j through an NST-stage ring
@@ -70,9 +69,7 @@ struct PrefillCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NST * TILE_BYTES;
-  static constexpr int MAX_LIST = 512;              // work items one CTA can be dealt
-  static constexpr int OFF_LIST = OFF_V + NST * TILE_BYTES;  // int [MAX_LIST] + count
-  static constexpr int OFF_BAR = OFF_LIST + (MAX_LIST + 16) * 4;
+  static constexpr int OFF_BAR = OFF_V + NST * TILE_BYTES;
   static constexpr int N_BARS = 2 + 4 * NST + 2 + 2 + 2 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
@@ -158,51 +155,6 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
   return it;
 }
 
-// The CTA's work items: the items with an active query row, in index order (heaviest causal query
-// tile first, so their tile counts do not increase), dealt to the CTAs in snake order — round r
-// goes to CTAs 0..grid-1 for even r and grid-1..0 for odd r — which keeps the CTAs' total work
-// within a tile or two of each other where a plain round robin leaves the heaviest CTA well above
-// the mean (packed batches with many empty items especially).  One warp builds the list with
-// ballots: item idx has rank k among the active items, and goes to round k / grid of CTA
-// snake(k % grid).  Returns the item count, or -1 when a CTA would be dealt more than MAX_LIST
-// items (then every CTA takes items blockIdx.x + i * gridDim.x instead).
-template <int MAXL>
-__device__ __forceinline__ int prefill_build_schedule(const PrefillParams& p, int* list, int lane) {
-  const int grid = gridDim.x, c = blockIdx.x;
-  int k = 0;
-  for (int base = 0; base < p.n_items; base += 32) {
-    const int idx = base + lane;
-    bool active = false;
-    if (idx < p.n_items) {
-      const PrefillItem it = prefill_item(p, idx);
-      active = it.active[0] || it.active[1];
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, active);
-    if (active) {
-      const int kk = k + __popc(bal & ((1u << lane) - 1u));
-      const int r = kk / grid, pos = kk - r * grid;
-      const int cta = (r & 1) ? grid - 1 - pos : pos;
-      if (cta == c && r < MAXL) list[r] = idx;
-    }
-    k += __popc(bal);
-  }
-  const int full = k / grid, rem = k - full * grid;
-  const int mine = full + (rem > ((full & 1) ? grid - 1 - c : c) ? 1 : 0);
-  return (k > MAXL * grid) ? -1 : mine;
-}
-
-// The CTA's item count and its i-th item: the dealt list, or every gridDim.x-th item when the list
-// would overflow (list[MAXL] holds the count, -1 for the fallback).
-template <int MAXL>
-__device__ __forceinline__ int prefill_items_mine(const PrefillParams& p, const int* list) {
-  const int n = list[MAXL];
-  return n >= 0 ? n : (p.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-}
-template <int MAXL>
-__device__ __forceinline__ int prefill_item_at(const int* list, int i) {
-  return list[MAXL] >= 0 ? list[i] : (int)blockIdx.x + i * (int)gridDim.x;
-}
-
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -253,11 +205,6 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
     if (lane == 0) ATTN_TRACE_AT(1, 2, 0);
   }
-  int* const list = reinterpret_cast<int*>(smem + C::OFF_LIST);
-  if (warp == 2) {
-    const int cnt = prefill_build_schedule<C::MAX_LIST>(p, list, lane);
-    if (lane == 0) list[C::MAX_LIST] = cnt;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -280,8 +227,7 @@ __global__ void __launch_bounds__(384, 1)
       int g = 0, qi = 0;  // tiles loaded, items with tiles
       int nk = 0, nv = 0;  // K / V tiles issued
       bool ok = true, q_pending = false;
-      for (int li = 0; li < prefill_items_mine<C::MAX_LIST>(p, list) && ok; ++li) {
-        const int idx = prefill_item_at<C::MAX_LIST>(list, li);
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const PrefillItem it = prefill_item(p, idx);
         const int n = it.n_tiles;
         if (n == 0) continue;
@@ -361,8 +307,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       int g = 0, qi = 0;
       bool ok = true;
-      for (int li = 0; li < prefill_items_mine<C::MAX_LIST>(p, list) && ok; ++li) {
-        const int idx = prefill_item_at<C::MAX_LIST>(list, li);
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int n = prefill_item(p, idx).n_tiles;
         if (n == 0) continue;
         if (lane == 0) ATTN_TRACE_AT(1, 3, qi);
@@ -444,8 +389,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tmem + 256 + slot * D + lane_off;
     int g = 0, qi = 0;
     bool ok = true;
-    for (int li = 0; li < prefill_items_mine<C::MAX_LIST>(p, list) && ok; ++li) {
-        const int idx = prefill_item_at<C::MAX_LIST>(list, li);
+    for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
       const PrefillItem it = prefill_item(p, idx);
       const int n = it.n_tiles;
       const int q_lo = it.q_lo[slot];

@@ -165,10 +165,9 @@ def test_prefill_strided_no_visible_keys(cuda_device):
     device_clean()
 
 
-def test_prefill_more_items_than_the_schedule_holds(cuda_device):
-    """80000 one-token sequences make 80000 work items, more than the 512 per CTA the kernel's
-    schedule list holds at 148 CTAs: every CTA falls back to taking every grid-th item, and every
-    row is still computed (one visible key: O = V, LSE = scale * q.k)."""
+def test_prefill_many_work_items(cuda_device):
+    """80000 one-token sequences make 80000 work items, 540 for each CTA of the persistent grid:
+    every row is computed (one visible key: O = V, LSE = scale * q.k)."""
     B, D = 80000, 64
     q, k, v = _gen(B, 1, 1, 1, 1, D, seed=25)
     o, lse = A.attn_prefill(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), causal=True)
