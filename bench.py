@@ -49,14 +49,14 @@ L2_BYTES = 126 * 10**6
 NCU_TRAFFIC = {
     "prefill": {"sources": ('ptx.cuh', 'status.cuh', 'prefill.cuh'), "sha1": "1f04feae59dccef5",
         "bytes": 319281920 + 103592448},
-    "decode_b4_h32g8_d128_ragged64k_128k": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh'), "sha1": "05bf10cb7a6761a8",
-        "bytes": 1549369000 + 4824320},
-    "decode_fp8_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_fp8.cuh'), "sha1": "3f42ea4af4db181d",
-        "bytes": 1147681000 + 5401088},
-    "decode_int8_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "fe9dc325b38c9ea7",
-        "bytes": 1147788000 + 5465856},
-    "decode_int4_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "fe9dc325b38c9ea7",
-        "bytes": 606726400 + 5503744},
+    "decode_b4_h32g8_d128_ragged64k_128k": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh'), "sha1": "6b6cf2c3fc7aa803",
+        "bytes": 1549382144 + 4482816},
+    "decode_fp8_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_fp8.cuh'), "sha1": "b3ac03fa062a074c",
+        "bytes": 1147788288 + 4960000},
+    "decode_int8_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "ba2b83f64c27b8e1",
+        "bytes": 1147688448 + 4968192},
+    "decode_int4_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "ba2b83f64c27b8e1",
+        "bytes": 607405568 + 4998912},
 }
 
 
