@@ -28,9 +28,10 @@
 //   warps 10..13 Q staging, softmax, epilogue: thread = token (later = output element d)
 // Issuing a tcgen05.mma costs its thread tens of cycles, so the S and PV chains (8 MMAs each per
 // tile) go to two threads, ordered only through barriers: S(j+NB) waits until the softmax has read
-// S(j) (s_free), and the softmax writes P(j+NB) once PV(j) has completed.  Scores, probabilities and
-// converted tiles rotate through NB = 3 buffers.  TMEM columns: S^T [0, 48) (three 16-column
-// buffers), O^T [48, 64), converted K [64, 256) (three 64-column buffers, 128 f16 per lane).
+// S(j) (s_free), and the softmax writes P(j+NB) once PV(j) has completed.  The softmax takes two
+// tiles per step; scores, probabilities and converted K rotate through NB = 4 buffers, converted V
+// through NV (4 for INT4, 3 for INT8).  TMEM columns: S^T [0, 64) (16-column buffers), O^T
+// [64, 80), converted K [128, 384) (64-column buffers, 128 f16 per lane).
 #pragma once
 
 #include "decode.cuh"
@@ -42,7 +43,13 @@ struct DecodeIntCfg {
   static constexpr int D = 128;
   static constexpr int ROW = BITS == 8 ? 128 : 64;  // code bytes per token row
   static constexpr int NCS = 3;                     // stages of raw code tiles
-  static constexpr int NB = 3;                      // S / P / converted-tile buffers
+  // The softmax runs over two tiles per step (one maxima exchange and rescale decision per 256
+  // tokens, up to eight query rows per KV head); S^T, P^T and converted K then rotate in fours.
+  // Converted V tiles (32 KB each) get four buffers for INT4 and three for INT8, whose raw code
+  // stages take twice the shared memory.
+  static constexpr int STEP = 2;
+  static constexpr int NB = 4;                      // S / P / converted-K buffers
+  static constexpr int NV = BITS == 4 ? 4 : 3;      // converted-V buffers
   static constexpr int CODE_TILE = 128 * ROW;
   static constexpr int VC_TILE = 2 * 128 * 128;     // 128 tokens x 128 f16, two 64-wide boxes
   static constexpr int QBOX = 16 * 128;             // 16 rows x 64 f16
@@ -52,16 +59,17 @@ struct DecodeIntCfg {
   static constexpr int OFF_KCODE = 0;
   static constexpr int OFF_VCODE = OFF_KCODE + NCS * CODE_TILE;
   static constexpr int OFF_VC = OFF_VCODE + NCS * CODE_TILE;
-  static constexpr int OFF_Q = OFF_VC + NB * VC_TILE;
+  static constexpr int OFF_Q = OFF_VC + NV * VC_TILE;
   static constexpr int OFF_P = OFF_Q + Q_BYTES;
   static constexpr int OFF_RED = OFF_P + NB * P_BYTES;
   static constexpr int OFF_QSC = OFF_RED + (2 * 4 * 16 + 4 * 16) * 4;  // [16] 2^-e per query row
   static constexpr int OFF_BAR = OFF_QSC + 16 * 4;
-  static constexpr int N_BARS = 4 * NCS + 1 + 8 * NB + 2 + 2 + 1 + 1;
+  static constexpr int N_BARS = 4 * NCS + 1 + 6 * NB + 2 * NV + 2 + 2 + 1 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
   static constexpr int THREADS = 512;
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t COL_S = 0, COL_O = 48, COL_K = 64;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_O = NB * 16, COL_K = 128;  // S^T, O^T, converted K
+  static_assert(COL_O + 16 <= COL_K && COL_K + NB * 64 <= TMEM_COLS, "TMEM columns");
   static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
 static_assert(DecodeIntCfg<8>::SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
@@ -196,43 +204,61 @@ __device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kv
   }
 }
 
-// One tile of the softmax on the thread that owns token t, with the running max over
-// y = x + log2(v_scale): row maxima (warp redux, then the cross-warp exchange) -> lazy O rescale
-// -> this token's entries of P^T (2^(y - m), f16).  Returns false, warp-uniformly, if a bounded
-// wait ran out.  The parities follow decode_softmax_core.
-// S^T of the tile is read first and s_free is arrived on at once, so the next S into the same
-// buffer can be issued; the P^T buffer is written only after p_reuse (the PV that last read it, if
-// any) has completed.
-template <int GP>
-__device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, int lane, int wq, int t, bool valid,
-                                                 const float (&scq)[GP], float ks, float vs, uint32_t tS_lane,
-                                                 uint64_t* s_free, uint32_t tO_lane, float* red_max,
+// One softmax step over NT tiles (one or, for INT4, two) on the thread that owns token t of each,
+// with the running max over y = x + log2(v_scale): row maxima over the step's tokens (warp redux,
+// then the cross-warp exchange number e) -> lazy O rescale -> this thread's entries of each tile's
+// P^T (2^(y - m), f16).  nt (warp-uniform) is how many of the NT tiles exist (the last step of an
+// odd tile count has one).  Returns false, warp-uniformly, if a bounded wait ran out.  The S^T of
+// every tile is read first and its s_free arrived on at once, so the next S into the same buffer
+// can be issued; a P^T buffer is written only after p_reuse (the PV that last read it, if any) has
+// completed.
+template <int GP, int NT>
+__device__ __forceinline__ bool int_softmax_step(DecodeRows<GP>& rows, int e, int j, int nt, int lane, int wq, int t,
+                                                 const bool (&valid)[NT], const float (&scq)[GP], const float (&ks)[NT],
+                                                 const float (&vs)[NT], const uint32_t (&tS_lane)[NT],
+                                                 uint64_t* const (&s_free)[NT], uint32_t tO_lane, float* red_max,
                                                  uint64_t* red_bar, uint64_t* prev_pv, uint32_t prev_pv_parity,
-                                                 uint64_t* p_reuse, uint32_t p_reuse_parity, uint8_t* p_tile,
-                                                 float threshold, long long* evt_base_ = nullptr) {
-  uint32_t sv[16];
-  tmem_ld16(tS_lane, sv);
-  tmem_wait_ld();
+                                                 uint64_t* const (&p_reuse)[NT], const uint32_t (&p_reuse_parity)[NT],
+                                                 uint8_t* const (&p_tile)[NT], float threshold,
+                                                 long long* evt_base_ = nullptr) {
+  uint32_t sv[NT][16];
+#pragma unroll
+  for (int k = 0; k < NT; ++k)
+    if (k < nt) tmem_ld16(tS_lane[k], sv[k]);
+#pragma unroll
+  for (int k = 0; k < NT; ++k)
+    if (k < nt) tmem_wait_ld_regs(sv[k]);
   if (t == 0) ATTN_EVT(j, 10);
   if (lane == 0 && j < 31) ATTN_EVT(32 + j, 4 + wq);
   tc_fence_before();
-  warp_arrive(s_free, lane);
-  const float avs = fminf(fmaxf(fabsf(vs), 0x1p-100f), 0x1p100f);
-  const float lvs = __log2f(avs);
-  const float ivs = __fdividef(1.f, avs);
-  const bool neg = vs < 0.f;
-  float y[GP];
 #pragma unroll
-  for (int g = 0; g < GP; ++g) y[g] = valid ? fmaf(__uint_as_float(sv[g]) * scq[g], ks, lvs) : -INFINITY;
-  float* rm = red_max + (j & 1) * 64;
+  for (int k = 0; k < NT; ++k)
+    if (k < nt) warp_arrive(s_free[k], lane);
+  float lvs[NT], ivs[NT];
+  bool neg[NT];
+  float y[NT][GP];
+#pragma unroll
+  for (int k = 0; k < NT; ++k) {
+    const float avs = fminf(fmaxf(fabsf(vs[k]), 0x1p-100f), 0x1p100f);
+    lvs[k] = __log2f(avs);
+    ivs[k] = __fdividef(1.f, avs);
+    neg[k] = vs[k] < 0.f;
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+      y[k][g] = (k < nt && valid[k]) ? fmaf(__uint_as_float(sv[k][g]) * scq[g], ks[k], lvs[k]) : -INFINITY;
+  }
+  float* rm = red_max + (e & 1) * 64;
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
-    const float m = warp_max_redux(y[g]);
+    float ym = y[0][g];
+#pragma unroll
+    for (int k = 1; k < NT; ++k) ym = fmaxf(ym, y[k][g]);
+    const float m = warp_max_redux(ym);
     if (lane == 0) rm[wq * 16 + g] = m;
   }
   if (lane == 0 && j < 31) ATTN_EVT(32 + j, wq);
-  warp_arrive(&red_bar[j & 1], lane);  // lane 0 wrote this warp's maxima
-  if (!mbar_wait_warp(&red_bar[j & 1], (j >> 1) & 1, SITE_DC_SM_S)) return false;
+  warp_arrive(&red_bar[e & 1], lane);  // lane 0 wrote this warp's maxima
+  if (!mbar_wait_warp(&red_bar[e & 1], (e >> 1) & 1, SITE_DC_SM_S)) return false;
   if (t == 0) ATTN_EVT(j, 11);
   bool need = false;
   float alpha[GP];
@@ -254,22 +280,28 @@ __device__ __forceinline__ bool int_softmax_tile(DecodeRows<GP>& rows, int j, in
     tc_fence_after();
     uint32_t orow[16];
     tmem_ld16(tO_lane, orow);
-    tmem_wait_ld();
+    tmem_wait_ld_regs(orow);
 #pragma unroll
     for (int g = 0; g < GP; ++g) orow[g] = __float_as_uint(__uint_as_float(orow[g]) * alpha[g]);
     tmem_st16(tO_lane, orow);
     tmem_wait_st();
   }
-  if (p_reuse && !mbar_wait_warp(p_reuse, p_reuse_parity, SITE_DC_SM_P)) return false;
+#pragma unroll
+  for (int k = 0; k < NT; ++k)
+    if (k < nt && p_reuse[k] && !mbar_wait_warp(p_reuse[k], p_reuse_parity[k], SITE_DC_SM_P)) return false;
   if (t == 0) ATTN_EVT(j, 12);
-  uint8_t* prow = p_tile + (t >> 6) * (16 * 128);
   const uint32_t pchunk = (t & 63) >> 3, pbyte = (t & 7) * 2;
 #pragma unroll
-  for (int g = 0; g < GP; ++g) {
-    const float pe = (y[g] == -INFINITY) ? 0.f : ex2_approx(y[g] - rows.m_used[g]);
-    rows.l_part[g] += pe * ivs;
-    *reinterpret_cast<uint16_t*>(prow + sw128_offset(g, pchunk) + pbyte) =
-        __half_as_ushort(__float2half_rn(neg ? -pe : pe));
+  for (int k = 0; k < NT; ++k) {
+    if (k >= nt) break;
+    uint8_t* prow = p_tile[k] + (t >> 6) * (16 * 128);
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float pe = (y[k][g] == -INFINITY) ? 0.f : ex2_approx(y[k][g] - rows.m_used[g]);
+      rows.l_part[g] += pe * ivs[k];
+      *reinterpret_cast<uint16_t*>(prow + sw128_offset(g, pchunk) + pbyte) =
+          __half_as_ushort(__float2half_rn(neg[k] ? -pe : pe));
+    }
   }
   return true;
 }
@@ -312,9 +344,9 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* pv_done = p_full + NB;   // [NB] PV(j) completed
   uint64_t* kc_full = pv_done + NB;  // [NB] converted K in TMEM
   uint64_t* kc_empty = kc_full + NB; // [NB] S MMA done reading it
-  uint64_t* vc_full = kc_empty + NB; // [NB] converted V in shared memory
-  uint64_t* vc_empty = vc_full + NB; // [NB] PV MMA done reading it
-  uint64_t* s_free = vc_empty + NB;  // [NB] the softmax has read S^T(j)
+  uint64_t* vc_full = kc_empty + NB;     // [NV] converted V in shared memory
+  uint64_t* vc_empty = vc_full + C::NV;  // [NV] PV MMA done reading it
+  uint64_t* s_free = vc_empty + C::NV;   // [NB] the softmax has read S^T(j)
   uint64_t* drain = s_free + NB;     // [2] each MMA issuer's own MMAs completed
   uint64_t* red_bar = drain + 2;     // [2]
   uint64_t* sum_bar = red_bar + 2;
@@ -338,9 +370,11 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&pv_done[s], 1);
       mbar_init(&kc_full[s], 4);
       mbar_init(&kc_empty[s], 1);
+      mbar_init(&s_free[s], 4);
+    }
+    for (int s = 0; s < C::NV; ++s) {
       mbar_init(&vc_full[s], 4);
       mbar_init(&vc_empty[s], 1);
-      mbar_init(&s_free[s], 4);
     }
     mbar_init(&red_bar[0], 4);
     mbar_init(&red_bar[1], 4);
@@ -418,21 +452,21 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t sP = smem_u32(smem + C::OFF_P);
         const uint32_t sVc = smem_u32(smem + C::OFF_VC);
         for (int j = 0; j < n && ok; ++j) {
-          const int bj = j % NB;
-          const uint32_t ph = (j / NB) & 1;
+          const int bj = j % NB, bv = j % C::NV;
+          const uint32_t ph = (j / NB) & 1, phv = (j / C::NV) & 1;
           ATTN_EVT(j, 8);
-          if (!(ok = mbar_wait(&vc_full[bj], ph, SITE_DC_MMA_V))) break;
+          if (!(ok = mbar_wait(&vc_full[bv], phv, SITE_DC_MMA_V))) break;
           ATTN_EVT(j, 9);
           if (!(ok = mbar_wait(&p_full[bj], ph, SITE_DC_MMA_P))) break;
           tc_fence_after();
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t da = make_sdesc_sw128(sVc + bj * C::VC_TILE + kk * 16 * 128, 128 * 128, 1024);
+            const uint64_t da = make_sdesc_sw128(sVc + bv * C::VC_TILE + kk * 16 * 128, 128 * 128, 1024);
             const uint64_t db = make_sdesc_sw128(sP + bj * C::P_BYTES + (kk >> 2) * C::PBOX + (kk & 3) * 32, 16, 1024);
             mma_ss(tO, da, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
           ATTN_EVT(j, 7);
           mma_commit(&pv_done[bj]);
-          mma_commit(&vc_empty[bj]);
+          mma_commit(&vc_empty[bv]);
         }
         if (ok) mma_commit(o_final);
         mma_commit(&drain[1]);
@@ -476,13 +510,13 @@ __global__ void __launch_bounds__(512, 1)
     for (int j = 0; j < n; ++j) {
       const int st = j % C::NCS;
       const uint32_t ph = (j / C::NCS) & 1;
-      const int bj = j % NB;
-      const uint32_t phb = (j / NB) & 1;
+      const int bv = j % C::NV;
+      const uint32_t phv = (j / C::NV) & 1;
       const bool valid = t0 + j * 128 + t < t1;
       if (!mbar_wait_warp(&v_full[st], ph, SITE_DC_SM_V)) break;
-      if (!mbar_wait_warp(&vc_empty[bj], phb ^ 1, SITE_DC_SM_V)) break;  // PV(j-NB) has read it
+      if (!mbar_wait_warp(&vc_empty[bv], phv ^ 1, SITE_DC_SM_V)) break;  // PV(j-NV) has read it
       const uint8_t* vtile = smem + C::OFF_VCODE + st * C::CODE_TILE;
-      uint8_t* vc = smem + C::OFF_VC + bj * C::VC_TILE;
+      uint8_t* vc = smem + C::OFF_VC + bv * C::VC_TILE;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {  // elements [64 half, +64) = box `half` of the operand
         uint32_t h[32];
@@ -496,7 +530,7 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&v_empty[st]);
-        mbar_arrive(&vc_full[bj]);
+        mbar_arrive(&vc_full[bv]);
       }
       if (t == 0) ATTN_EVT(j, 3);
     }
@@ -542,47 +576,75 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    for (int j = 0; j < n && ok; ++j) {
-      const int bj = j % NB;
-      const uint32_t phb = (j / NB) & 1;
-      const int tok = t0 + j * 128 + t;
-      const bool valid = tok < t1;
-      const float ks = ksr[0], vs = vsr[0];
+    // Sixteen query rows per KV head hold twice the scores per tile: their step stays one tile wide
+    // so both tiles' rows need not be live at once.
+    constexpr int ST = GP <= 8 ? C::STEP : 1;
+    for (int j = 0; j < n && ok; j += ST) {
+      const int nt = n - j < ST ? n - j : ST;  // tiles in this step (warp-uniform)
+      bool valid[ST];
+      float ks[ST], vs[ST];
+      uint32_t tSl[ST], prp[ST];
+      uint64_t* sfr[ST];
+      uint64_t* prb[ST];
+      uint8_t* ptl[ST];
 #pragma unroll
-      for (int i = 0; i + 1 < SPF; ++i) {
-        ksr[i] = ksr[i + 1];
-        vsr[i] = vsr[i + 1];
+      for (int k = 0; k < ST; ++k) {
+        const int jk = j + k;
+        const int bk = jk % NB;
+        valid[k] = t0 + jk * 128 + t < t1;
+        ks[k] = ksr[k];
+        vs[k] = vsr[k];
+        tSl[k] = tS0 + bk * 16 + lane_off;
+        sfr[k] = &s_free[bk];
+        // PV(i) is completion number i/NB of pv_done[i%NB]; PV(jk-NB), the last reader of P buffer
+        // bk, is the oldest pending phase of its barrier (PV(jk) needs this step's P first).
+        prb[k] = jk >= NB ? &pv_done[bk] : nullptr;
+        prp[k] = ((uint32_t)(jk / NB) & 1) ^ 1;
+        ptl[k] = smem + C::OFF_P + bk * C::P_BYTES;
       }
-      ksr[SPF - 1] = 1.f;
-      vsr[SPF - 1] = 1.f;
-      if (tok + SPF * 128 < t1) {
-        const long long x = int_scale_index(p, b, tok + SPF * 128, kvh);
-        if (x >= 0) {
-          ksr[SPF - 1] = __ldg(p.k_scale + x);
-          vsr[SPF - 1] = __ldg(p.v_scale + x);
+      // Per-token scales: the ring holds SPF tiles; this step consumes ST of them and refills the
+      // same number SPF tiles ahead.
+#pragma unroll
+      for (int i = 0; i + ST < SPF; ++i) {
+        ksr[i] = ksr[i + ST];
+        vsr[i] = vsr[i + ST];
+      }
+#pragma unroll
+      for (int k = 0; k < ST; ++k) {
+        const int tk = t0 + (j + k + SPF) * 128 + t;
+        ksr[SPF - ST + k] = 1.f;
+        vsr[SPF - ST + k] = 1.f;
+        if (tk < t1) {
+          const long long x = int_scale_index(p, b, tk, kvh);
+          if (x >= 0) {
+            ksr[SPF - ST + k] = __ldg(p.k_scale + x);
+            vsr[SPF - ST + k] = __ldg(p.v_scale + x);
+          }
         }
       }
       if (t == 0) ATTN_EVT(j, 13);
       if (lane == 0 && j < 31) ATTN_EVT(32 + j, 8 + wq);
-      if (!(ok = mbar_wait_warp(&s_full[bj], phb, SITE_DC_SM_S))) break;
+#pragma unroll
+      for (int k = 0; k < ST; ++k)
+        if (k < nt && !(ok = mbar_wait_warp(&s_full[(j + k) % NB], (uint32_t)((j + k) / NB) & 1, SITE_DC_SM_S))) break;
+      if (!ok) break;
       if (t == 0) ATTN_EVT(j, 5);
       tc_fence_after();
-      // PV(i) is completion number i/NB of pv_done[i%NB]; PV(j-1) and PV(j-NB) (the last reader of
-      // P buffer bj) are the oldest pending phases of their barriers, since PV(j) and later need
-      // this tile's P first, so each parity wait is unambiguous.
+      // PV(j-1) is the oldest pending phase of its barrier (PV(j-1+NB) needs a later P).
       const int jp = j > 0 ? j - 1 : 0;
-      if (!(ok = int_softmax_tile<GP>(rows, j, lane, wq, t, valid, scq, ks, vs, tS0 + bj * 16 + lane_off,
-                                      &s_free[bj], tO + lane_off, red_max, red_bar, &pv_done[jp % NB],
-                                      (uint32_t)(jp / NB) & 1, j >= NB ? &pv_done[bj] : nullptr, phb ^ 1,
-                                      smem + C::OFF_P + bj * C::P_BYTES, C::RESCALE_THRESHOLD
+      if (!(ok = int_softmax_step<GP, ST>(rows, j / ST, j, nt, lane, wq, t, valid, scq, ks, vs, tSl, sfr,
+                                          tO + lane_off, red_max, red_bar, &pv_done[jp % NB],
+                                          (uint32_t)(jp / NB) & 1, prb, prp, ptl, C::RESCALE_THRESHOLD
 #ifdef ATTN_PROF
-                                      , evt_base_
+                                          , evt_base_
 #endif
-                                      )))
+                                          )))
         break;
       fence_proxy_async_smem();
       tc_fence_before();
-      warp_arrive(&p_full[bj], lane);
+#pragma unroll
+      for (int k = 0; k < ST; ++k)
+        if (k < nt) warp_arrive(&p_full[(j + k) % NB], lane);
       if (t == 0) ATTN_EVT(j, 6);
       if (lane == 0 && j < 31) ATTN_EVT(32 + j, 12 + wq);
     }

@@ -23,6 +23,7 @@ def _run(d, dev, splits=0):
     o, lse = A.attn_decode_splitkv(d["q"].to(dev), d["k_codes"].to(dev), d["v_codes"].to(dev), d["kv_lens"].to(dev),
                                    k_scale=d["k_scale"].to(dev), v_scale=d["v_scale"].to(dev), num_splits=splits)
     torch.cuda.synchronize()
+    device_clean()  # a wait that ran out leaves stale partials: report it as such, not as a mismatch
     return o, lse
 
 
@@ -53,6 +54,27 @@ def test_int_groups(cuda_device, bits, Hq, Hkv):
         ro, rl = _ref(d, w.scale)
         assert_o_close(o, ro)
         assert_lse_close(lse, rl)
+    device_clean()
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (64, 8), (48, 4)])
+def test_int_many_items_per_cta(cuda_device, bits, Hq, Hkv):
+    """More (split, KV head, sequence) work items than SMs, so each persistent CTA walks several,
+    with empty splits, single tokens and odd tile counts between them."""
+    g = torch.Generator().manual_seed(bits * 100 + Hq + Hkv)
+    lens = torch.randint(0, 1537, (48,), generator=g)
+    lens[::7] = 0
+    lens[3::11] = 1
+    lens[5::13] = 1536
+    w, d = _case(lens.tolist(), 1536, bits, Hq=Hq, Hkv=Hkv, seed=900 + bits + Hq)
+    ro, rl = _ref(d, w.scale)
+    for splits in (3, 0):
+        o, lse = _run(d, cuda_device, splits)
+        assert_o_close(o, ro)
+        assert_lse_close(lse, rl)
+        empty = (d["kv_lens"] == 0).nonzero().flatten().tolist()
+        assert all(torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b])) for b in empty)
     device_clean()
 
 
