@@ -176,3 +176,32 @@ def test_prefill_many_work_items(cuda_device):
     assert_o_close(o, ro)
     assert_lse_close(to_np(lse).transpose(0, 2, 1), rl)
     device_clean()
+
+
+def test_prefill_concurrent_streams(cuda_device):
+    """Three launches in flight at once on three streams (persistent grids sharing the SMs, each
+    walking its own work items): all match the oracle."""
+    cases = [_gen(1, 1024, 1024, 8, 2, 128, seed=31), _gen(2, 640, 640, 4, 4, 64, seed=32),
+             _gen(1, 384, 384, 2, 1, 128, seed=33)]
+    dev_cases = [tuple(x.to(cuda_device) for x in c) for c in cases]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    outs = []
+    for (q, k, v), s in zip(dev_cases, streams):
+        with torch.cuda.stream(s):
+            outs.append(A.attn_prefill(q, k, v, causal=True, stream=s))
+    torch.cuda.synchronize()
+    for (q, k, v), (o, lse) in zip(cases, outs):
+        ro, rl = O.attention(q, k, v, scale=1 / math.sqrt(q.shape[-1]), causal=True)
+        assert_o_close(o, ro)
+        assert_lse_close(to_np(lse).transpose(0, 2, 1), rl)
+    device_clean()
+
+
+def test_prefill_alternating_head_sizes(cuda_device):
+    """Launches of the D = 64 and D = 128 kernels interleaved in one process: every row is computed
+    each time (no state carries from one launch or instantiation to the next)."""
+    cases = [_gen(1, 300, 300, 8, 2, 64, seed=41), _gen(1, 300, 300, 8, 2, 128, seed=42)]
+    for _ in range(3):
+        for q, k, v in cases:
+            _check(q, k, v, cuda_device, causal=True)
