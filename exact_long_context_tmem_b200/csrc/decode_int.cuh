@@ -6,15 +6,18 @@
 // elements per byte, element 2i in the low nibble of byte i (a 128-element row is 64 bytes).  Each
 // (token, KV head) has one float32 scale for K and one for V; value = code * scale.
 //
-// The dequantisation is fused into the tile load.  TMA brings the raw code tiles into shared
-// memory; converter warps widen them to f16 (exact: every INT8 and INT4 value is an f16 value) -- K
-// straight into TMEM as the A operand of S^T = K . Q^T, V into shared memory as the A operand of
-// O^T += V^T . P^T -- and the scales stay out of the operands: k_scale multiplies the token's score
-// and v_scale its probability, on the thread that owns the token.
-//
-// Q is one f16 row per query head, scaled by a power of two 2^e that puts the row's absmax in
-// [2^14, 2^15): every bf16 element within 2^31 of the row max is then an exact f16, and the score
-// is S_mma * 2^-e.  The running max is taken over y = x + log2(v_scale) (x the log2-domain score),
+// The dequantisation is fused into the tile load, and the scales stay out of the operands: k_scale
+// multiplies the token's score and v_scale its probability, on the thread that owns the token.
+// TMA brings the raw code tiles into shared memory.
+//  * Scores, INT8: the K code tile is, as it lands, the K-major A operand of an integer MMA
+//    (kind::i8, int32 accumulation) against Q as three signed 8-bit digits per element: the row
+//    scaled by 2^e (absmax in [2^21, 2^22)) and rounded, q = 65536 d0 + 256 d1 + d2; the softmax
+//    recombines the three digit columns exactly, so the score is (K . q) 2^-e with no conversion of
+//    K at all.
+//  * Scores, INT4: converter warps widen K to f16 (exact) straight into TMEM, the A operand of
+//    S^T = K . Q^T, against Q as one f16 row per head scaled by 2^e (absmax in [2^14, 2^15)).
+//  * Values (both): converter warps widen V to f16 in shared memory, the MN-major A operand of
+//    O^T += V^T . P^T.  The running max is taken over y = x + log2(v_scale) (x the log2-domain score),
 // so the probability that enters P, 2^(y - m) = 2^(x - m) * v_scale, stays below 2^threshold
 // whatever the scale; the row sum l adds 2^(x - m) = P / v_scale.
 //
@@ -23,7 +26,7 @@
 //   warp 14      TMA producer of the raw V code tiles (NCS-stage ring)
 //   warp 1       TMEM allocator; lane 0 issues the S MMAs
 //   warp 15      lane 0 issues the PV MMAs
-//   warps 2..5   K converter: thread = token; codes -> f16 into TMEM
+//   warps 2..5   K converter (INT4): thread = token; codes -> f16 into TMEM
 //   warps 6..9   V converter: thread = token; codes -> f16 in shared memory (MN-major operand)
 //   warps 10..13 Q staging, softmax, epilogue: thread = token (later = output element d)
 // Issuing a tcgen05.mma costs its thread tens of cycles, so the S and PV chains (8 MMAs each per
@@ -53,7 +56,10 @@ struct DecodeIntCfg {
   static constexpr int CODE_TILE = 128 * ROW;
   static constexpr int VC_TILE = 2 * 128 * 128;     // 128 tokens x 128 f16, two 64-wide boxes
   static constexpr int QBOX = 16 * 128;             // 16 rows x 64 f16
-  static constexpr int Q_BYTES = 2 * QBOX;
+  // INT8: the score MMA takes the K codes as TMA lands them (kind::i8) against Q as three signed
+  // 8-bit digits per element (up to 48 rows of 128 bytes); INT4: Q as f16 rows (two boxes).
+  static constexpr bool K_I8 = BITS == 8;
+  static constexpr int Q_BYTES = K_I8 ? 48 * 128 : 2 * QBOX;
   static constexpr int PBOX = 16 * 128;
   static constexpr int P_BYTES = 2 * PBOX;
   static constexpr int OFF_KCODE = 0;
@@ -68,8 +74,10 @@ struct DecodeIntCfg {
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16 + 1024;
   static constexpr int THREADS = 512;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S = 0, COL_O = NB * 16, COL_K = 128;  // S^T, O^T, converted K
-  static_assert(COL_O + 16 <= COL_K && COL_K + NB * 64 <= TMEM_COLS, "TMEM columns");
+  // S^T from column 0 (NB buffers of 16 columns, or for INT8 of 16 / 32 / 48: three digit columns
+  // per query row), O^T at 64 (INT4) or 256 (INT8), converted K (INT4) from 128.
+  static constexpr uint32_t COL_S = 0, COL_O = K_I8 ? 256 : NB * 16, COL_K = 128;
+  static_assert(K_I8 ? NB * 48 <= (int)COL_O : (COL_O + 16 <= COL_K && COL_K + NB * 64 <= TMEM_COLS), "TMEM columns");
   static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
 static_assert(DecodeIntCfg<8>::SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
@@ -96,6 +104,53 @@ __device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t& h01, uint32_t&
   const uint32_t u = w ^ 0x80808080u;
   h01 = sub_f16x2(__byte_perm(u, 0x64646464u, 0x5150u), 0x64806480u);
   h23 = sub_f16x2(__byte_perm(u, 0x64646464u, 0x5352u), 0x64806480u);
+}
+
+// INT8 scores on the tensor core: S^T = K codes . Q digits^T with int32 accumulation (kind::i8,
+// K = 32 per instruction).  Instruction descriptor: s32 accumulator (format 2 at bit 4), A and B
+// signed 8-bit (format 1 at bits 7 and 10), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t make_idesc_s8(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_s8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// S^T columns per buffer for a group padded to GP rows: 16, or for INT8 3 GP digit columns
+// rounded up to 16.
+template <int GP, int BITS>
+__host__ __device__ constexpr int int_score_cols() {
+  return BITS == 8 ? ((3 * GP + 15) / 16) * 16 : 16;
+}
+
+// N consecutive TMEM columns of this warp's lanes (N = 16, 32 or 48), waited for.
+template <int N>
+__device__ __forceinline__ void int_tmem_ld(uint32_t taddr, uint32_t (&v)[N]) {
+  static_assert(N == 16 || N == 32 || N == 48, "column count");
+  if constexpr (N == 16) {
+    tmem_ld16(taddr, v);
+    tmem_wait_ld_regs(v);
+  } else if constexpr (N == 32) {
+    tmem_ld32(taddr, v);
+    tmem_wait_ld_regs(v);
+  } else {
+    uint32_t a[32], b[16];
+    tmem_ld32(taddr, a);
+    tmem_ld16(taddr + 32, b);
+    tmem_wait_ld_regs(a);
+    tmem_wait_ld_regs(b);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = a[c];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) v[32 + c] = b[c];
+  }
 }
 
 __device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t b, uint32_t c) {
@@ -166,11 +221,17 @@ __device__ __forceinline__ long long int_scale_index(const DecodeParams& p, int 
   return (page * p.page_size + off) * p.Hkv + kvh;
 }
 
-// Query rows of the group as f16 rows scaled by 2^e (absmax in [2^14, 2^15); e clamped to
-// [-100, 100]) into the 128B-swizzled K-major B operand (two 64-wide boxes of 16 rows); 2^-e of
-// row g goes to qsc[g].  128 threads: chunk c = tid + 128 k is row c / 16, elements 8 (c % 16)..,
-// so the 16 threads of a row are 16 consecutive lanes of one warp.
-template <int BITS>
+// Query rows of the group, staged as the B operand of the score MMA; 2^-e of row g goes to qsc[g].
+// 128 threads: chunk c = tid + 128 k is row c / 16, elements 8 (c % 16).., so the 16 threads of a
+// row are 16 consecutive lanes of one warp, which find the row's absmax together.
+//  INT4: f16 rows scaled by 2^e (absmax in [2^14, 2^15); every bf16 element within 2^31 of it is
+//    then exact) into the 128B-swizzled K-major operand (two 64-wide boxes of 16 rows), elements in
+//    the paired order of the widened K rows.
+//  INT8: integers q = rn(x 2^e) with the absmax in [2^21, 2^22) (exact for every element within
+//    2^14 of it), written as three balanced signed 8-bit digits q = 65536 d0 + 256 d1 + d2
+//    (|d0| <= 64): digit k of row g is operand row k GP + g, one 128-byte row of 128 elements.
+//  e is clamped to [-100, 100].
+template <int BITS, int GP>
 __device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kvh, int b, int tid, uint8_t* q_smem,
                                             float* qsc) {
 #pragma unroll
@@ -189,17 +250,38 @@ __device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kv
     }
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    int e = 14 - ((int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127);
+    int e = (BITS == 8 ? 21 : 14) - ((int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127);
     e = e < -100 ? -100 : (e > 100 ? 100 : e);
     const float up = __uint_as_float((uint32_t)(e + 127) << 23);
-    uint32_t hv[4];
+    if constexpr (BITS == 8) {
+      uint32_t dw[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (BITS == 8) hv[i] = pack_f16x2(f[2 * i] * up, f[2 * i + 1] * up);
-      else hv[i] = pack_f16x2(f[i] * up, f[i + 4] * up);  // the paired order of the INT4 K rows
+      for (int i = 0; i < 8; ++i) {
+        const int q = __float2int_rn(f[i] * up);
+        const int d2 = ((q + 128) & 255) - 128;
+        const int r = (q - d2) >> 8;
+        const int d1 = ((r + 128) & 255) - 128;
+        const int d0 = (r - d1) >> 8;
+        const int sh = 8 * (i & 3);
+        dw[0][i >> 2] |= ((uint32_t)d0 & 0xFFu) << sh;
+        dw[1][i >> 2] |= ((uint32_t)d1 & 0xFFu) << sh;
+        dw[2][i >> 2] |= ((uint32_t)d2 & 0xFFu) << sh;
+      }
+      if (g < GP) {
+#pragma unroll
+        for (int dk = 0; dk < 3; ++dk) {
+          const uint32_t row = (uint32_t)(dk * GP + g);
+          *reinterpret_cast<uint2*>(q_smem + row * 128u + ((((uint32_t)cc >> 1) ^ (row & 7u)) << 4) +
+                                    ((uint32_t)cc & 1u) * 8u) = make_uint2(dw[dk][0], dw[dk][1]);
+        }
+      }
+    } else {
+      uint32_t hv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) hv[i] = pack_f16x2(f[i] * up, f[i + 4] * up);  // the paired order of the K rows
+      *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * (16 * 128) + sw128_offset(g, cc & 7)) =
+          make_uint4(hv[0], hv[1], hv[2], hv[3]);
     }
-    *reinterpret_cast<uint4*>(q_smem + (cc >> 3) * (16 * 128) + sw128_offset(g, cc & 7)) =
-        make_uint4(hv[0], hv[1], hv[2], hv[3]);
     if (cc == 0) qsc[g] = __uint_as_float((uint32_t)(127 - e) << 23);
   }
 }
@@ -212,7 +294,7 @@ __device__ __forceinline__ void int_stage_q(const DecodeParams& p, int G, int kv
 // every tile is read first and its s_free arrived on at once, so the next S into the same buffer
 // can be issued; a P^T buffer is written only after p_reuse (the PV that last read it, if any) has
 // completed.
-template <int GP, int NT>
+template <int GP, int NT, int BITS>
 __device__ __forceinline__ bool int_softmax_step(DecodeRows<GP>& rows, int e, int j, int nt, int lane, int wq, int t,
                                                  const bool (&valid)[NT], const float (&scq)[GP], const float (&ks)[NT],
                                                  const float (&vs)[NT], const uint32_t (&tS_lane)[NT],
@@ -221,13 +303,20 @@ __device__ __forceinline__ bool int_softmax_step(DecodeRows<GP>& rows, int e, in
                                                  uint64_t* const (&p_reuse)[NT], const uint32_t (&p_reuse_parity)[NT],
                                                  uint8_t* const (&p_tile)[NT], float threshold,
                                                  long long* evt_base_ = nullptr) {
-  uint32_t sv[NT][16];
+  constexpr int SC = int_score_cols<GP, BITS>();
+  uint32_t sv[NT][SC];
+  if constexpr (SC == 16) {
 #pragma unroll
-  for (int k = 0; k < NT; ++k)
-    if (k < nt) tmem_ld16(tS_lane[k], sv[k]);
+    for (int k = 0; k < NT; ++k)
+      if (k < nt) tmem_ld16(tS_lane[k], sv[k]);
 #pragma unroll
-  for (int k = 0; k < NT; ++k)
-    if (k < nt) tmem_wait_ld_regs(sv[k]);
+    for (int k = 0; k < NT; ++k)
+      if (k < nt) tmem_wait_ld_regs(sv[k]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < NT; ++k)
+      if (k < nt) int_tmem_ld<SC>(tS_lane[k], sv[k]);
+  }
   if (t == 0) ATTN_EVT(j, 10);
   if (lane == 0 && j < 31) ATTN_EVT(32 + j, 4 + wq);
   tc_fence_before();
@@ -244,8 +333,14 @@ __device__ __forceinline__ bool int_softmax_step(DecodeRows<GP>& rows, int e, in
     ivs[k] = __fdividef(1.f, avs);
     neg[k] = vs[k] < 0.f;
 #pragma unroll
-    for (int g = 0; g < GP; ++g)
-      y[k][g] = (k < nt && valid[k]) ? fmaf(__uint_as_float(sv[k][g]) * scq[g], ks[k], lvs[k]) : -INFINITY;
+    for (int g = 0; g < GP; ++g) {
+      float raw;  // Q.K of row g in units of 2^-e
+      if constexpr (BITS == 8)  // digits: 65536 S0 + (256 S1 + S2), each partial an exact int32
+        raw = fmaf((float)(int)sv[k][g], 65536.f, (float)((int)sv[k][GP + g] * 256 + (int)sv[k][2 * GP + g]));
+      else
+        raw = __uint_as_float(sv[k][g]);
+      y[k][g] = (k < nt && valid[k]) ? fmaf(raw * scq[g], ks[k], lvs[k]) : -INFINITY;
+    }
   }
   float* rm = red_max + (e & 1) * 64;
 #pragma unroll
@@ -359,7 +454,7 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NCS; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 4);
+      mbar_init(&k_empty[i], C::K_I8 ? 1 : 4);  // the S MMA's commit, or the K converter warps
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 4);
     }
@@ -425,7 +520,30 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------------ MMA issuers (S: warp 1, PV: warp 15)
     if (lane == 0) {
       bool ok = true;
-      if (warp == 1) {
+      if (warp == 1 && C::K_I8) {
+        // S^T(j) [128 x SC] = K codes_j (as TMA landed them) . Q digits^T, int32 (4 steps of 32
+        // codes); the commit after it frees the raw K stage.
+        constexpr int SC = int_score_cols<GP, BITS>();
+        constexpr uint32_t idesc_qk = make_idesc_s8(128, SC);
+        const uint32_t sQ = smem_u32(smem + C::OFF_Q), sK = smem_u32(smem + C::OFF_KCODE);
+        ok = mbar_wait(q_ready, 0, SITE_DC_MMA_K);
+        for (int j = 0; j < n && ok; ++j) {
+          const int bj = j % NB, st = j % C::NCS;
+          const uint32_t ph = (j / NB) & 1;
+          if (!(ok = mbar_wait(&k_full[st], (j / C::NCS) & 1, SITE_DC_MMA_K))) break;
+          if (j >= NB && !(ok = mbar_wait(&s_free[bj], ph ^ 1, SITE_DC_MMA_S))) break;  // S(j-NB) read
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_s8_ss(tS0 + bj * SC, make_sdesc_sw128(sK + st * C::CODE_TILE + kk * 32, 16, 1024),
+                      make_sdesc_sw128(sQ + kk * 32, 16, 1024), idesc_qk, kk > 0);
+          ATTN_EVT(j, 4);
+          mma_commit(&s_full[bj]);
+          mma_commit(&k_empty[st]);
+        }
+        mma_commit(&drain[0]);
+        mbar_wait_drain(&drain[0], 0, SITE_DC_DRAIN);
+      } else if (warp == 1) {
         // S^T(j) [128 x 16] = K_j (TMEM, f16) . Q^T
         constexpr uint32_t idesc_qk = make_idesc_f16(128, 16, false, false, false);
         const uint32_t sQ = smem_u32(smem + C::OFF_Q);
@@ -476,10 +594,11 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp < 6) {
     // ------------------------------------------------------------------ K converter warpgroup
+    // (INT4 only: the INT8 score MMA reads the codes directly)
     const int wq = warp & 3;
     const int t = wq * 32 + lane;  // token row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < (C::K_I8 ? 0 : n); ++j) {
       const int st = j % C::NCS;
       const uint32_t ph = (j / C::NCS) & 1;
       const int bj = j % NB;
@@ -542,7 +661,10 @@ __global__ void __launch_bounds__(512, 1)
     const int wg_tid = threadIdx.x - 320;
     for (int i = wg_tid; i < NB * C::P_BYTES / 16; i += 128)  // P^T rows >= GP stay zero
       reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
-    int_stage_q<BITS>(p, G, kvh, b, wg_tid, smem + C::OFF_Q, qsc);
+    if constexpr (C::K_I8)  // operand rows past the 3 GP digit rows stay zero
+      for (int i = 3 * GP * 128 / 16 + wg_tid; i < C::Q_BYTES / 16; i += 128)
+        reinterpret_cast<uint4*>(smem + C::OFF_Q)[i] = make_uint4(0u, 0u, 0u, 0u);
+    int_stage_q<BITS, GP>(p, G, kvh, b, wg_tid, smem + C::OFF_Q, qsc);
     fence_proxy_async_smem();
     warp_arrive(q_ready, lane);
     named_barrier_sync(1, 128);  // every row's 2^-e is in qsc
@@ -576,9 +698,9 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    // Sixteen query rows per KV head hold twice the scores per tile: their step stays one tile wide
-    // so both tiles' rows need not be live at once.
-    constexpr int ST = GP <= 8 ? C::STEP : 1;
+    // Groups whose tile scores fill 32 or more columns (16 rows; 8 rows of INT8 digits) keep a
+    // one-tile step, so two tiles' scores need not be live at once.
+    constexpr int ST = int_score_cols<GP, BITS>() * GP <= 128 && GP <= 8 ? C::STEP : 1;
     for (int j = 0; j < n && ok; j += ST) {
       const int nt = n - j < ST ? n - j : ST;  // tiles in this step (warp-uniform)
       bool valid[ST];
@@ -594,7 +716,7 @@ __global__ void __launch_bounds__(512, 1)
         valid[k] = t0 + jk * 128 + t < t1;
         ks[k] = ksr[k];
         vs[k] = vsr[k];
-        tSl[k] = tS0 + bk * 16 + lane_off;
+        tSl[k] = tS0 + bk * int_score_cols<GP, BITS>() + lane_off;
         sfr[k] = &s_free[bk];
         // PV(i) is completion number i/NB of pv_done[i%NB]; PV(jk-NB), the last reader of P buffer
         // bk, is the oldest pending phase of its barrier (PV(jk) needs this step's P first).
@@ -632,7 +754,7 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_after();
       // PV(j-1) is the oldest pending phase of its barrier (PV(j-1+NB) needs a later P).
       const int jp = j > 0 ? j - 1 : 0;
-      if (!(ok = int_softmax_step<GP, ST>(rows, j / ST, j, nt, lane, wq, t, valid, scq, ks, vs, tSl, sfr,
+      if (!(ok = int_softmax_step<GP, ST, BITS>(rows, j / ST, j, nt, lane, wq, t, valid, scq, ks, vs, tSl, sfr,
                                           tO + lane_off, red_max, red_bar, &pv_done[jp % NB],
                                           (uint32_t)(jp / NB) & 1, prb, prp, ptl, C::RESCALE_THRESHOLD
 #ifdef ATTN_PROF
