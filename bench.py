@@ -53,10 +53,10 @@ NCU_TRAFFIC = {
         "bytes": 1549382144 + 4482816},
     "decode_fp8_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_fp8.cuh'), "sha1": "b3ac03fa062a074c",
         "bytes": 1147788288 + 4960000},
-    "decode_int8_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "da94caa2da46bbbd",
-        "bytes": 1147226624 + 5640704},
-    "decode_int4_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "da94caa2da46bbbd",
-        "bytes": 609820928 + 4911104},
+    "decode_int8_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "ea38a1d9e25a36f6",
+        "bytes": 1147653376 + 5013760},
+    "decode_int4_b16_h32g8_d128_t32768": {"sources": ('ptx.cuh', 'status.cuh', 'decode.cuh', 'decode_int.cuh'), "sha1": "ea38a1d9e25a36f6",
+        "bytes": 601052928 + 4892416},
 }
 
 
