@@ -100,6 +100,28 @@ def test_int_scale_extremes(cuda_device, bits):
 
 
 @pytest.mark.parametrize("bits", [8, 4])
+def test_int_query_dynamic_range(cuda_device, bits):
+    """Query rows whose elements span 2^-30 .. 2^2 of one large element, a row with a single
+    nonzero element, and an all-zero row: the INT8 scores take Q as integers of 22 bits (elements
+    below 2^-14 of the row maximum are rounded), the INT4 scores as scaled f16 rows."""
+    w, d = _case([1500, 900], 1500, bits, Hq=16, Hkv=4, seed=121)
+    g = torch.Generator().manual_seed(7)
+    q = d["q"].float()
+    span = torch.pow(2.0, torch.randint(-30, 3, q.shape, generator=g).float())
+    q = q * span
+    q[0, 1] = 0.0
+    q[0, 1, 17] = 3.0
+    q[1, 2] = 0.0
+    d["q"] = q.to(torch.bfloat16)
+    for splits in (1, 2):
+        o, lse = _run(d, cuda_device, splits)
+        ro, rl = _ref(d, w.scale)
+        assert_o_close(o, ro)
+        assert_lse_close(lse, rl)
+    device_clean()
+
+
+@pytest.mark.parametrize("bits", [8, 4])
 def test_int_all_code_values(cuda_device, bits):
     """Every code value (-128..127 / -8..7) appears in K and V, at both ends of a row."""
     w, d = _case([640], 640, bits, Hq=8, Hkv=1, seed=97)
